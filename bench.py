@@ -1,0 +1,380 @@
+#!/usr/bin/env python
+"""Benchmark of one absorbed-MLA decode step on B200, through the C ABI.
+
+A step is one pass of the whole decode path over one batch of synthetic input:
+  mla_cache_append (RoPE on the new keys + paged scatter),
+  mla_absorb_q (W^UK folded into the query, RoPE on q^R),
+  mla_decode_attention (split-KV attention + log-sum-exp combine),
+  mla_out_absorb (W^UV applied to the latent output).
+Default workload: DeepSeek-V3-shaped decode, 64 sequences x 4096 cached tokens,
+128 heads, one query token each ("v3").
+
+Prints one JSON line (rank 0). Multi-GPU (torchrun): every rank runs its own
+replica of the workload (the path shards by sequence with no exchange), the
+device time is the max over ranks and ``value`` counts all ranks' tokens.
+
+``--impl reference`` times the CPU fp64 oracle (the only reference that exists
+for this method) on the host cores, on a bounded sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MLA decode tokens/sec and cache GB/s (% of HBM/bf16 roofline) on 1 B200"
+UNIT = "tokens/s"
+ROW_BYTES = 1152                 # 576 bf16 per cached token
+FLOP_PER_TOKEN_HEAD = 2 * 576 + 2 * 512
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# DRAM traffic per launch of mla_decode_attention measured by ncu
+# (dram__bytes_read.sum + dram__bytes_write.sum), keyed by the SHA-256 of the
+# decode sources it was measured on; reported only while the sources match.
+TRAFFIC = {}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--workload", default="v3")
+    ap.add_argument("--num-ctas", type=int, default=0)
+    ap.add_argument("--max-split", type=int, default=0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def decode_sources_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "mla_latent_kv_32_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.startswith("decode") or name in ("plan.h", "common.cuh"):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+class ClockSampler:
+    """Samples nvidia-smi SM clocks and throttle reasons while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+            time.sleep(0.25)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            if self.thread:
+                self.thread.join(timeout=2)
+
+    def summary(self):
+        if not self.lines:
+            return None
+        mhz, max_mhz, reasons, power = [], 0.0, set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                mhz.append(float(parts[1]))
+                max_mhz = max(max_mhz, float(parts[2]))
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not mhz:
+            return None
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": max_mhz,
+                "reasons": sorted(reasons), "samples": len(mhz),
+                "power_w_max": max(power) if power else None}
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def oracle_sample(w, inp, budget_s=12.0, max_seqs=None):
+    """Time the absorbed fp64 oracle on whole sequences of the workload until
+    ~budget_s of CPU work (at least one sequence). Returns (tokens/s, desc)."""
+    from oracle import mla_oracle as O
+    table = O.rope_table(int(inp.lens.max()))
+    scale = 1.0 / math.sqrt(192)
+    done, t_tot, cache_bytes = 0, 0.0, 0
+    order = list(range(w.B))
+    for b in order:
+        L = int(inp.lens[b])
+        n_pref = L - w.q_len
+        prefix = (O.gather_rows(inp.pool, inp.table, b, n_pref) if n_pref > 0
+                  else np.zeros((0, 576), np.uint16))
+        t0 = time.perf_counter()
+        O.decode_sequence(prefix, inp.c_new[b], inp.k_new[b], inp.q_nope[b], inp.q_pe[b],
+                          inp.w_uk, inp.w_uv, L, table, scale)
+        t_tot += time.perf_counter() - t0
+        done += 1
+        cache_bytes += L * ROW_BYTES
+        if t_tot >= budget_s or (max_seqs and done >= max_seqs):
+            break
+    tokens = done * w.q_len
+    desc = (f"absorbed fp64 oracle (numpy), {done} of {w.B} sequences of workload "
+            f"'{w.name}' ({tokens} query tokens, {cache_bytes / 1e6:.1f} MB of cache rows), "
+            f"{t_tot:.2f} s")
+    return tokens / t_tot, desc, t_tot
+
+
+def run_reference(args, rank, world):
+    import synth
+    if rank != 0:
+        return 0
+    w = synth.WORKLOADS[args.workload]
+    inp = synth.make_decode_inputs(w)
+    per_step = []
+    desc = ""
+    budget = max(1.0, 120.0 / max(1, args.steps + args.warmup))
+    for s in range(args.warmup + args.steps):
+        tps, desc, t = oracle_sample(w, inp, budget_s=budget)
+        if s >= args.warmup:
+            per_step.append(tps)
+    v = statistics.median(per_step)
+    cores = cpu_threads()
+    out = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": None,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(w, inp, None),
+        "cpu_baseline": {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+    return 0
+
+
+def workload_config(w, inp, sess):
+    cfg = {"workload": f"{w.name}: absorbed MLA decode, batch {w.B}, {w.q_len} query token(s) "
+                       f"per sequence, context {'U[1,%d]' % w.L if w.lens == 'ragged' else w.L}, "
+                       f"n_h {w.n_h}, d_c 512, d_R 64, paged cache of 64-token pages",
+           "batch": w.B, "q_len": w.q_len, "n_h": w.n_h,
+           "context_tokens": int(inp.lens.sum()),
+           "cache_bytes": int(inp.lens.sum()) * ROW_BYTES,
+           "l2": "flushed between timed steps (256 MiB write, outside the step events)"}
+    if sess is not None:
+        cfg["plan"] = {"work_lists": int(sess.info.num_ctas), "items": int(sess.info.num_items),
+                       "partials": int(sess.info.num_partials)}
+    return cfg
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    import torch
+    import torch.distributed as dist
+    import synth
+    from mla_latent_kv_32_b200 import build as build_mod
+    from mla_latent_kv_32_b200 import mla
+    from mla_latent_kv_32_b200.runtime import DecodeSession
+
+    assert torch.cuda.is_available(), "bench.py needs a CUDA device"
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    if rank == 0 or not os.path.exists(mla.LIB_PATH):
+        build_mod.build()
+    if world > 1:
+        dist.barrier()
+    mla.load()
+
+    w = synth.WORKLOADS[args.workload]
+    assert not w.layer, "bench.py times the attention-only decode workloads"
+    inp = synth.make_decode_inputs(w)
+    sess = DecodeSession(inp, dev, num_ctas=args.num_ctas, max_split=args.max_split)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(max(3, args.warmup)):
+        sess.step()
+    torch.cuda.synchronize()
+    bits = sess.read_status()
+    assert bits == 0, f"device status 0x{bits:x} during warm-up"
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    with ClockSampler(local) as clocks:
+        barrier()
+        for k in range(K):
+            flush.zero_()
+            e = ev[k]
+            e[0].record(stream)
+            sess.append()
+            sess.absorb()
+            e[1].record(stream)
+            sess.attend()
+            e[2].record(stream)
+            sess.expand()
+            e[3].record(stream)
+        barrier()
+    step_ms = [e[0].elapsed_time(e[3]) for e in ev]
+    attn_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    t_step = sum(step_ms) / K
+    t_attn = sum(attn_ms) / K
+    if world > 1:
+        t = torch.tensor([t_step, t_attn], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        t_step, t_attn = float(t[0]), float(t[1])
+
+    tokens = w.B * w.q_len
+    value = world * tokens / (t_step / 1e3)
+    cache_bytes = int(inp.lens.sum()) * ROW_BYTES
+    # FLOPs: 2176 per (visible cached token, head, query)
+    vis = sum(int(L) - w.q_len + j + 1 for L in inp.lens for j in range(w.q_len))
+    flops = float(vis) * w.n_h * FLOP_PER_TOKEN_HEAD
+
+    # e2e: per-step inputs from pinned host memory, result read back
+    e2e = None
+    if not args.no_e2e:
+        ins, host_in, host_out = sess.pinned_step_buffers()
+        h2d, d2h = DecodeSession.step_io_bytes(ins, host_out)
+        for _ in range(3):
+            sess.step_e2e(ins, host_in, host_out)
+        torch.cuda.synchronize()
+        ee = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(K)]
+        barrier()
+        for k in range(K):
+            flush.zero_()
+            ee[k][0].record(stream)
+            sess.step_e2e(ins, host_in, host_out)
+            ee[k][1].record(stream)
+        barrier()
+        t_e2e = sum(a.elapsed_time(b) for a, b in ee) / K
+        if world > 1:
+            t = torch.tensor([t_e2e], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            t_e2e = float(t[0])
+        e2e = {"value": world * tokens / (t_e2e / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "ms_per_step": t_e2e}
+
+    peaks, peak_src = load_peaks()
+    gbs = cache_bytes / (t_attn / 1e3) / 1e9
+    tfs = flops / (t_attn / 1e3) / 1e12
+    t_mem = cache_bytes / (peaks["hbm_gbs"] * 1e9)
+    t_tc = flops / (peaks["bf16_tflops"] * 1e12)
+    src_hash = decode_sources_hash()
+    traffic = TRAFFIC.get(src_hash)
+    roof = {
+        "kernel": "mla_decode_attention (decode + combine kernels)",
+        "bound": "hbm" if t_mem >= t_tc else "tensor",
+        "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+        "frac": gbs / peaks["hbm_gbs"], "traffic": traffic,
+        "algorithmic_bytes": cache_bytes, "algorithmic_flops": flops,
+        "tensor": {"achieved": tfs, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                   "frac": tfs / peaks["bf16_tflops"]},
+        "roofline_us": max(t_mem, t_tc) * 1e6, "measured_us": t_attn * 1e3,
+        "frac_of_roofline": max(t_mem, t_tc) / (t_attn / 1e3),
+        "peak_source": f"{peak_src} (MEASURED_PEAKS.json burst figures)"
+        if peak_src == "measured" else "fallback", "sources": src_hash,
+    }
+    # cache_append, absorb GEMM, q RoPE pack, decode, [combine], out_absorb
+    launches_per_step = 5 + (1 if sess.info.num_combine > 0 else 0)
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": t_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": workload_config(w, inp, sess),
+        "cache_gbs": cache_bytes / (t_step / 1e3) / 1e9 * world,
+        "attention_ms": t_attn,
+        "roofline": roof,
+        "e2e": e2e,
+        "gpu_launches": launches_per_step * K,
+        "clocks": clocks.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu:
+        tps, desc, _ = oracle_sample(w, inp, budget_s=12.0)
+        out["cpu_baseline"] = {"value": tps, "unit": UNIT, "cores": cpu_threads(),
+                               "kind": "oracle", "sample": desc}
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,243 @@
+/*
+ * mla.h -- C ABI of the absorbed Multi-Head Latent Attention (MLA) decode
+ * library for NVIDIA B200 (sm_100a).
+ *
+ * The library computes one decode step of MLA with weight absorption over a
+ * paged latent cache, as described on the MLA pages:
+ *   - the cache holds, per token, the 512-dim latent c^KV and the 64-dim
+ *     decoupled RoPE key k^R ("DeepSeek-V3 MLA: Multi-Head Latent Attention
+ *     Guide", section "4. Cache Footprint Math");
+ *   - W^UK is folded into the query, q~_i = (W^UK_i)^T q^C_i, and the scores
+ *     are taken directly on the latents, score_j = q~_i . c_j + q^R_i . k^R_j
+ *     (same page, "The Matrix Absorption Trick", part 2);
+ *   - the softmax-weighted latents o_i = sum_j a_ij c_j are expanded once
+ *     through W^UV, u_i = W^UV_i o_i (same page, part 3).
+ *
+ * Conventions shared by every call:
+ *   - All tensors are caller-owned. Pointers documented as "device" must be
+ *     device memory of the current CUDA device; "host" pointers are host
+ *     memory. The library allocates no device memory in any call.
+ *   - bf16 tensors are passed as uint16_t bit patterns (mla_bf16_t).
+ *   - Every device call is asynchronous on the given stream (a cudaStream_t
+ *     passed as void*; NULL = the legacy default stream) and never
+ *     synchronises, except mla_read_status.
+ *   - Every call returns an mla_status_t; no C++ exception crosses the ABI.
+ *     On an error nothing is launched (argument errors) and a message is
+ *     available from mla_last_error() on the calling thread.
+ *   - Kernels that find bad data (a page id outside the pool, a position
+ *     outside the RoPE table, an expired bounded wait) skip the affected
+ *     work and OR an MLA_DEV_* bit into the optional device status word
+ *     `status` (a uint32_t in device memory, may be NULL). They never trap.
+ *   - Device pointers must be 16-byte aligned unless stated otherwise; row
+ *     strides (in elements) must keep every row 16-byte aligned.
+ */
+#ifndef MLA_H_
+#define MLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t mla_bf16_t;   /* bf16 bit pattern */
+typedef void *mla_stream_t;    /* cudaStream_t */
+
+/* Fixed widths of the method (DeepSeek-V2/V3 MLA). */
+#define MLA_D_C 512    /* latent width of c^KV */
+#define MLA_D_R 64     /* decoupled RoPE width of k^R, q^R */
+#define MLA_D_NOPE 128 /* per-head content query/key width d_h */
+#define MLA_D_V 128    /* per-head value width */
+#define MLA_ROW 576    /* cached elements per token: [c^KV | k^R] */
+#define MLA_PAGE 64    /* tokens per cache page */
+
+typedef enum mla_status {
+  MLA_OK = 0,
+  MLA_ERR_INVALID_ARGUMENT = 1,    /* null/misaligned pointer, bad size or stride */
+  MLA_ERR_UNSUPPORTED = 2,         /* shape outside the supported set, or not sm_100 */
+  MLA_ERR_WORKSPACE_TOO_SMALL = 3, /* plan or workspace buffer smaller than required */
+  MLA_ERR_CUDA = 4,                /* a CUDA runtime/driver call failed */
+  MLA_ERR_DEVICE = 5               /* mla_read_status found device status bits set */
+} mla_status_t;
+
+/* Device status bits (OR-ed into the caller's status word). */
+#define MLA_DEV_BAD_PAGE 0x1u     /* page id or sequence index out of range: work skipped */
+#define MLA_DEV_BAD_POSITION 0x2u /* position outside the RoPE table or the page table */
+#define MLA_DEV_TIMEOUT 0x4u      /* a bounded wait expired: the kernel abandoned its work */
+#define MLA_DEV_BAD_PLAN 0x8u     /* a work item disagrees with the sequence lengths */
+
+/* Message of the last failed call on this thread ("" if none). */
+const char *mla_last_error(void);
+
+/* Library ABI version (increments on any signature change). */
+int mla_version(void);
+
+/*
+ * mla_rope_table -- host. Fills table[max_pos][32][2] (float32) with
+ * (cos, sin) of theta_j = pos / base^(2j/64), j = 0..31, computed in double
+ * precision and rounded once to float. Interleaved pairs (2j, 2j+1) are
+ * rotated by theta_j ("Deconstructing DeepSeek V4 Pro ...", section "Hands-On
+ * PyTorch Implementation", apply_rope).
+ *   table: host, caller-owned, max_pos * 64 floats.
+ * Errors: INVALID_ARGUMENT if table is NULL, max_pos <= 0 or base <= 1.
+ */
+mla_status_t mla_rope_table(float *table, int max_pos, double base);
+
+/*
+ * mla_cache_append -- device. Appends n_tokens new tokens to the paged cache:
+ * for token t (sequence seq_idx[t], position pos[t]) the row
+ *   [c_kv[t][0:512] | RoPE(k_pe[t][0:64], pos[t])]
+ * is written to page block_table[seq_idx[t] * max_pages + pos[t] / 64],
+ * slot pos[t] % 64. The decoupled RoPE key is rotated before it is cached
+ * ("DeepSeek-V3 MLA ... Guide", "3. The Decoupled RoPE Key"; "Step 3" appends
+ * the new latent and rotated key to the cache before attention).
+ * The rotation is float32 with no fused multiply-add: for pair j,
+ *   y0 = x0*cos - x1*sin, y1 = x1*cos + x0*sin, each product and sum rounded
+ * once, then rounded to bf16 (nearest even), so the stored code is a fixed
+ * function of the inputs and the table.
+ *   cache:       device bf16 [num_pages][64][576], updated in place.
+ *   block_table: device int32 [batch][max_pages], page ids.
+ *   seq_idx,pos: device int32 [n_tokens].
+ *   c_kv:        device bf16, row t at c_kv + t*ld_c (512 elements).
+ *   k_pe:        device bf16, row t at k_pe + t*ld_k (64 elements, pre-RoPE).
+ *   rope_table:  device float32 [max_pos][32][2] (see mla_rope_table).
+ *   status:      device uint32 or NULL.
+ * A token with seq_idx outside [0,batch), pos outside [0,max_pos) or
+ * pos/64 >= max_pages, or whose page id is outside [0,num_pages), is skipped
+ * and sets MLA_DEV_BAD_PAGE / MLA_DEV_BAD_POSITION.
+ */
+mla_status_t mla_cache_append(mla_bf16_t *cache, int num_pages,
+                              const int32_t *block_table, int batch, int max_pages,
+                              const int32_t *seq_idx, const int32_t *pos,
+                              const mla_bf16_t *c_kv, int ld_c,
+                              const mla_bf16_t *k_pe, int ld_k,
+                              const float *rope_table, int max_pos, int n_tokens,
+                              uint32_t *status, mla_stream_t stream);
+
+/*
+ * mla_absorb_q -- device. Folds W^UK into the content query and packs the
+ * query row the attention kernel reads:
+ *   q_full[t][h][0:512]   = sum_d q_nope[t][h][d] * w_uk[h][d][:]
+ *   q_full[t][h][512:576] = RoPE(q_pe[t][h][:], pos[t])   (or a copy if pos == NULL)
+ * ("DeepSeek-V3 MLA ... Guide", "The Matrix Absorption Trick", part 2:
+ * q~ = (W^UK_i)^T q^C_i, computed once per query token).
+ *   q_nope: device bf16, element (t,h,d) at q_nope + t*ld_qn + h*128 + d.
+ *   q_pe:   device bf16, element (t,h,r) at q_pe + t*ld_qp + h*64 + r (pre-RoPE).
+ *   w_uk:   device bf16 [n_h][128][512] (the view(n_h, d_h, d_c) of W^UK).
+ *   pos:    device int32 [T] absolute positions, or NULL.
+ *   rope_table: device float32 [max_pos][32][2] (unused when pos == NULL).
+ *   q_full: device bf16 [T][n_h][576], written.
+ * fp32 accumulation, one bf16 rounding per output element.
+ * Supported: 1 <= n_h <= 128, n_h % 16 == 0.
+ */
+mla_status_t mla_absorb_q(const mla_bf16_t *q_nope, int ld_qn,
+                          const mla_bf16_t *q_pe, int ld_qp,
+                          const mla_bf16_t *w_uk, const int32_t *pos,
+                          const float *rope_table, int max_pos, int T, int n_h,
+                          mla_bf16_t *q_full, uint32_t *status, mla_stream_t stream);
+
+/*
+ * Decode plan. The split of each sequence's pages into work items is made on
+ * the host from the sequence lengths (split-KV: long sequences are cut into
+ * several items whose partial results are merged by a log-sum-exp combine).
+ * The plan is a flat byte buffer; its size depends only on (batch, q_len,
+ * num_ctas) and is returned by mla_plan_bytes. The caller copies the host plan
+ * to device memory (cudaMemcpyAsync) and passes both to mla_decode_attention.
+ */
+typedef struct mla_plan_info {
+  int num_items;        /* work items in the plan */
+  int num_ctas;         /* concurrent work lists (CTA clusters) the plan targets */
+  int num_partials;     /* partial-result slots used by split items */
+  int num_combine;      /* (sequence, query) pairs that need the combine pass */
+  size_t plan_bytes;    /* bytes of the plan actually used */
+  size_t workspace_bytes; /* device scratch mla_decode_attention needs */
+} mla_plan_info_t;
+
+/* Upper bound of the plan size for these sizes (host, no side effects). */
+size_t mla_plan_bytes(int batch, int q_len, int num_ctas);
+
+/*
+ * mla_decode_plan -- host.
+ *   seq_lens: host int32 [batch], total tokens of each sequence including the
+ *             q_len new ones (1 <= q_len <= seq_lens[b]).
+ *   num_ctas: work lists to balance over; 0 = derive from the current
+ *             device's SM count.
+ *   max_split: upper bound on the items one (sequence, query) is cut into; 0 = no bound.
+ *   plan:     host buffer of plan_bytes (>= mla_plan_bytes(batch, q_len, num_ctas)).
+ *   info:     out, may be NULL.
+ * Errors: INVALID_ARGUMENT (bad lengths), WORKSPACE_TOO_SMALL (plan buffer).
+ */
+mla_status_t mla_decode_plan(const int32_t *seq_lens, int batch, int q_len, int n_h,
+                             int num_ctas, int max_split, void *plan, size_t plan_bytes,
+                             mla_plan_info_t *info);
+
+/*
+ * mla_decode_attention -- device. Absorbed attention over the paged cache:
+ * for sequence b, query j (position p = L_b - q_len + j) and head h,
+ *   s_i   = (q_full[b][j][h][0:512] . c_i + q_full[b][j][h][512:576] . k^R_i) * scale,
+ *           for cached tokens i <= p (the new tokens are already appended);
+ *   a     = softmax(s);  o_latent[b][j][h][:] = sum_i a_i c_i;
+ *   lse[b][j][h] = log(sum_i exp(s_i)) (natural log), if lse != NULL.
+ * ("DeepSeek-V3 MLA ... Guide", "The Matrix Absorption Trick" parts 2-4 and
+ * "Step 3": scores on the 512-dim latents plus the RoPE term, softmax, latent
+ * output.) Long sequences are split across CTA clusters per the plan and
+ * merged by a log-sum-exp combine pass.
+ *   q_full:      device bf16 [batch][q_len][n_h][576] (from mla_absorb_q).
+ *   cache:       device bf16 [num_pages][64][576].
+ *   block_table: device int32 [batch][max_pages].
+ *   plan_host / plan_dev: the same plan bytes in host and device memory.
+ *   workspace:   device scratch of >= info.workspace_bytes (16-byte aligned).
+ *   o_latent:    device bf16 [batch][q_len][n_h][512], written.
+ *   lse:         device float32 [batch][q_len][n_h] or NULL.
+ * Cache slots past a sequence's length (inside its last page) must hold
+ * finite values: they are read, and given weight zero.
+ * Supported: n_h % 16 == 0, 16 <= n_h <= 128, 1 <= q_len <= 2.
+ */
+mla_status_t mla_decode_attention(const mla_bf16_t *q_full, const mla_bf16_t *cache,
+                                  int num_pages, const int32_t *block_table, int max_pages,
+                                  int batch, int q_len, int n_h, float scale,
+                                  const void *plan_host, const void *plan_dev,
+                                  void *workspace, size_t workspace_bytes,
+                                  mla_bf16_t *o_latent, float *lse, uint32_t *status,
+                                  mla_stream_t stream);
+
+/*
+ * mla_out_absorb -- device. Expands the latent attention output through W^UV:
+ *   u[t][h*128 + d] = sum_c o_latent[t][h][c] * w_uv[h][d][c]
+ * ("DeepSeek-V3 MLA ... Guide", "The Matrix Absorption Trick", part 3:
+ * u_i = W^UV_i o_i; "Step 3", einsum 'bnc,nhc->bnh').
+ *   o_latent: device bf16 [T][n_h][512].
+ *   w_uv:     device bf16 [n_h][128][512].
+ *   u:        device bf16, row t at u + t*ld_u (n_h*128 elements), written.
+ * fp32 accumulation, one bf16 rounding per output element.
+ */
+mla_status_t mla_out_absorb(const mla_bf16_t *o_latent, const mla_bf16_t *w_uv, int T,
+                            int n_h, mla_bf16_t *u, int ld_u, mla_stream_t stream);
+
+/*
+ * mla_gemm_bf16 -- device. Plain projection GEMM used by the decode layer
+ * (W^DQ, [W^UQ|W^QR], [W^DKV|W^KR], W^O; "DeepSeek-V3 MLA ... Guide",
+ * "Core Architecture & Mathematics" sections 1-2, and the output projection):
+ *   C[m][n] = sum_k X[m][k] * W[n][k]
+ *   X: device bf16 [M][K], row stride ld_x.  W: device bf16 [N][K] (nn.Linear
+ *   layout), row stride ld_w.  C: device, row stride ld_c, bf16 if c_fp32 == 0
+ *   else float32. fp32 accumulation.
+ */
+mla_status_t mla_gemm_bf16(const mla_bf16_t *X, int ld_x, const mla_bf16_t *W, int ld_w,
+                           void *C, int ld_c, int c_fp32, int M, int N, int K,
+                           mla_stream_t stream);
+
+/*
+ * mla_read_status -- host. Synchronises `stream`, copies the device status
+ * word to *bits and, if clear != 0, zeroes it. Returns MLA_ERR_DEVICE if any
+ * bit was set, MLA_OK otherwise.
+ */
+mla_status_t mla_read_status(uint32_t *status, uint32_t *bits, int clear,
+                             mla_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_H_ */

@@ -1,0 +1,399 @@
+// Host side of the C ABI: argument validation, the split-KV planner, the RoPE
+// table, status handling, and the launch sequence of each entry point.
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <algorithm>
+#include <mutex>
+#include <queue>
+#include <vector>
+
+#include "internal.h"
+
+namespace mla {
+
+static thread_local char g_err[1024];
+
+mla_status_t fail(mla_status_t st, const char *fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+void clear_error() { g_err[0] = '\0'; }
+
+mla_status_t device_info(int *num_sms, int *cc_major, int *cc_minor) {
+  static std::mutex mu;
+  static int cached[64][3];
+  static bool have[64] = {};
+  int dev = 0;
+  MLA_CUDA_TRY(cudaGetDevice(&dev));
+  std::lock_guard<std::mutex> lock(mu);
+  if (dev < 0 || dev >= 64) return fail(MLA_ERR_UNSUPPORTED, "device index %d", dev);
+  if (!have[dev]) {
+    MLA_CUDA_TRY(cudaDeviceGetAttribute(&cached[dev][0], cudaDevAttrMultiProcessorCount, dev));
+    MLA_CUDA_TRY(cudaDeviceGetAttribute(&cached[dev][1], cudaDevAttrComputeCapabilityMajor, dev));
+    MLA_CUDA_TRY(cudaDeviceGetAttribute(&cached[dev][2], cudaDevAttrComputeCapabilityMinor, dev));
+    have[dev] = true;
+  }
+  if (num_sms) *num_sms = cached[dev][0];
+  if (cc_major) *cc_major = cached[dev][1];
+  if (cc_minor) *cc_minor = cached[dev][2];
+  return MLA_OK;
+}
+
+static mla_status_t require_sm100() {
+  int major = 0, minor = 0;
+  mla_status_t st = device_info(nullptr, &major, &minor);
+  if (st != MLA_OK) return st;
+  if (major != 10)
+    return fail(MLA_ERR_UNSUPPORTED, "compute capability %d.%d: this library is built for sm_100a",
+                major, minor);
+  return MLA_OK;
+}
+
+static bool heads_supported(int n_h) { return n_h >= 16 && n_h <= 128 && n_h % 16 == 0; }
+
+// ---------------------------------------------------------------- planner ---
+
+static size_t align16(size_t x) { return (x + 15) & ~(size_t)15; }
+
+static size_t plan_bytes_for(int batch, int q_len, int num_ctas) {
+  const size_t units = (size_t)batch * q_len;
+  const size_t max_items = units + (size_t)num_ctas;
+  return sizeof(PlanHeader) + align16(sizeof(int32_t) * (num_ctas + 1)) +
+         max_items * sizeof(WorkItem) + units * sizeof(CombineItem);
+}
+
+static mla_status_t resolve_ctas(int *num_ctas) {
+  if (*num_ctas > 0) return MLA_OK;
+  int sms = 0;
+  mla_status_t st = device_info(&sms, nullptr, nullptr);
+  if (st != MLA_OK) return st;
+  *num_ctas = std::max(1, sms / 2);  // one CTA pair (cluster of 2) per work list
+  return MLA_OK;
+}
+
+}  // namespace mla
+
+using namespace mla;
+
+extern "C" {
+
+const char *mla_last_error(void) { return g_err; }
+
+int mla_version(void) { return 1; }
+
+mla_status_t mla_rope_table(float *table, int max_pos, double base) {
+  clear_error();
+  MLA_CHECK_ARG(table != nullptr, "rope table pointer is NULL");
+  MLA_CHECK_ARG(max_pos > 0, "max_pos must be positive (got %d)", max_pos);
+  MLA_CHECK_ARG(base > 1.0, "RoPE base must exceed 1 (got %g)", base);
+  double denom[MLA_D_R / 2];
+  for (int j = 0; j < MLA_D_R / 2; ++j) denom[j] = pow(base, 2.0 * j / MLA_D_R);
+  for (int p = 0; p < max_pos; ++p) {
+    for (int j = 0; j < MLA_D_R / 2; ++j) {
+      const double th = (double)p / denom[j];
+      table[(size_t)p * MLA_D_R + 2 * j] = (float)cos(th);
+      table[(size_t)p * MLA_D_R + 2 * j + 1] = (float)sin(th);
+    }
+  }
+  return MLA_OK;
+}
+
+mla_status_t mla_cache_append(mla_bf16_t *cache, int num_pages, const int32_t *block_table,
+                              int batch, int max_pages, const int32_t *seq_idx,
+                              const int32_t *pos, const mla_bf16_t *c_kv, int ld_c,
+                              const mla_bf16_t *k_pe, int ld_k, const float *rope_table,
+                              int max_pos, int n_tokens, uint32_t *status,
+                              mla_stream_t stream) {
+  clear_error();
+  MLA_CHECK_ARG(n_tokens >= 0, "n_tokens < 0");
+  if (n_tokens == 0) return MLA_OK;
+  MLA_CHECK_ARG(cache && block_table && seq_idx && pos && c_kv && k_pe && rope_table,
+                "NULL device pointer");
+  MLA_CHECK_ARG(num_pages > 0 && batch > 0 && max_pages > 0 && max_pos > 0,
+                "sizes must be positive");
+  MLA_CHECK_ARG(aligned16(cache) && aligned16(c_kv) && aligned16(k_pe) && aligned16(rope_table),
+                "cache, c_kv, k_pe and rope_table must be 16-byte aligned");
+  MLA_CHECK_ARG(ld_c >= MLA_D_C && ld_c % 8 == 0, "ld_c must be >= 512 and a multiple of 8");
+  MLA_CHECK_ARG(ld_k >= MLA_D_R && ld_k % 8 == 0, "ld_k must be >= 64 and a multiple of 8");
+  mla_status_t st = require_sm100();
+  if (st != MLA_OK) return st;
+  return launch_cache_append(cache, num_pages, block_table, batch, max_pages, seq_idx, pos,
+                             c_kv, ld_c, k_pe, ld_k, rope_table, max_pos, n_tokens, status,
+                             (cudaStream_t)stream);
+}
+
+mla_status_t mla_absorb_q(const mla_bf16_t *q_nope, int ld_qn, const mla_bf16_t *q_pe,
+                          int ld_qp, const mla_bf16_t *w_uk, const int32_t *pos,
+                          const float *rope_table, int max_pos, int T, int n_h,
+                          mla_bf16_t *q_full, uint32_t *status, mla_stream_t stream) {
+  clear_error();
+  MLA_CHECK_ARG(T >= 0, "T < 0");
+  if (T == 0) return MLA_OK;
+  if (!heads_supported(n_h))
+    return fail(MLA_ERR_UNSUPPORTED, "n_h = %d (supported: 16..128, multiple of 16)", n_h);
+  MLA_CHECK_ARG(q_nope && q_pe && w_uk && q_full, "NULL device pointer");
+  MLA_CHECK_ARG(pos == nullptr || (rope_table != nullptr && max_pos > 0),
+                "pos given without a RoPE table");
+  MLA_CHECK_ARG(aligned16(q_nope) && aligned16(q_pe) && aligned16(w_uk) && aligned16(q_full) &&
+                    (rope_table == nullptr || aligned16(rope_table)),
+                "pointers must be 16-byte aligned");
+  MLA_CHECK_ARG(ld_qn >= n_h * MLA_D_NOPE && ld_qn % 8 == 0, "ld_qn too small or unaligned");
+  MLA_CHECK_ARG(ld_qp >= n_h * MLA_D_R && ld_qp % 8 == 0, "ld_qp too small or unaligned");
+  mla_status_t st = require_sm100();
+  if (st != MLA_OK) return st;
+  st = launch_absorb_q(q_nope, ld_qn, w_uk, T, n_h, q_full, (cudaStream_t)stream);
+  if (st != MLA_OK) return st;
+  return launch_q_rope_pack(q_pe, ld_qp, pos, rope_table, max_pos, T, n_h, q_full, status,
+                            (cudaStream_t)stream);
+}
+
+size_t mla_plan_bytes(int batch, int q_len, int num_ctas) {
+  if (batch < 0 || q_len < 0) return 0;
+  if (resolve_ctas(&num_ctas) != MLA_OK) return 0;
+  return plan_bytes_for(batch, q_len, num_ctas);
+}
+
+mla_status_t mla_decode_plan(const int32_t *seq_lens, int batch, int q_len, int n_h,
+                             int num_ctas, int max_split, void *plan, size_t plan_bytes,
+                             mla_plan_info_t *info) {
+  clear_error();
+  MLA_CHECK_ARG(batch >= 0, "batch < 0");
+  MLA_CHECK_ARG(q_len >= 1 && q_len <= 2, "q_len must be 1 or 2 (got %d)", q_len);
+  if (!heads_supported(n_h))
+    return fail(MLA_ERR_UNSUPPORTED, "n_h = %d (supported: 16..128, multiple of 16)", n_h);
+  MLA_CHECK_ARG(batch == 0 || seq_lens != nullptr, "seq_lens is NULL");
+  MLA_CHECK_ARG(plan != nullptr, "plan is NULL");
+  MLA_CHECK_ARG(max_split >= 0, "max_split < 0");
+  mla_status_t st = resolve_ctas(&num_ctas);
+  if (st != MLA_OK) return st;
+  const size_t need = plan_bytes_for(batch, q_len, num_ctas);
+  if (plan_bytes < need)
+    return fail(MLA_ERR_WORKSPACE_TOO_SMALL, "plan buffer %zu B < %zu B", plan_bytes, need);
+  for (int b = 0; b < batch; ++b)
+    MLA_CHECK_ARG(seq_lens[b] >= q_len, "seq_lens[%d] = %d < q_len = %d", b, seq_lens[b], q_len);
+
+  // (b, j) units and their page counts: query j sees tokens 0..L-q_len+j.
+  struct Unit { int b, j, pages, L, qpos; };
+  std::vector<Unit> units;
+  units.reserve((size_t)batch * q_len);
+  long long total = 0;
+  int max_unit = 0;
+  for (int b = 0; b < batch; ++b)
+    for (int j = 0; j < q_len; ++j) {
+      const int L = seq_lens[b];
+      const int qpos = L - q_len + j;
+      const int pages = (qpos + 1 + MLA_PAGE - 1) / MLA_PAGE;
+      units.push_back({b, j, pages, L, qpos});
+      total += pages;
+      max_unit = std::max(max_unit, pages);
+    }
+  // Work lists. With max_split == 1 every (sequence, query) is one item and
+  // items go to lists by longest-processing-time order. Otherwise the units'
+  // pages are laid end to end and cut into num_ctas near-equal ranges, so
+  // every list carries the same page count; a unit crossing a cut becomes
+  // several items whose partial results the combine pass merges. Adjacent
+  // units (the two queries of an MTP step) start on neighbouring lists at the
+  // same time, so their shared pages are read once from HBM and once from L2.
+  std::vector<std::vector<WorkItem>> per;
+  std::vector<CombineItem> comb;
+  int slots = 0;
+  int max_pages_used = 0;
+  for (const Unit &u : units) max_pages_used = std::max(max_pages_used, u.pages);
+  if (max_split == 1) {
+    std::vector<int> order(units.size());
+    for (size_t i = 0; i < order.size(); ++i) order[i] = (int)i;
+    std::stable_sort(order.begin(), order.end(),
+                     [&](int x, int y) { return units[x].pages > units[y].pages; });
+    const int lists = std::max(1, std::min<int>(num_ctas, (int)units.size()));
+    typedef std::pair<long long, int> Load;
+    std::priority_queue<Load, std::vector<Load>, std::greater<Load>> heap;
+    for (int c = 0; c < lists; ++c) heap.push({0, c});
+    per.assign(lists, {});
+    for (int idx : order) {
+      const Unit &u = units[idx];
+      Load ld = heap.top();
+      heap.pop();
+      per[ld.second].push_back(WorkItem{u.b, u.j, 0, u.pages, -1, u.L, u.qpos, 0});
+      ld.first += u.pages;
+      heap.push(ld);
+    }
+  } else {
+    const int lists = (int)std::max<long long>(1, std::min<long long>(num_ctas, total));
+    const long long target = (total + lists - 1) / lists;
+    per.assign(lists, {});
+    int c = 0;
+    long long fill = 0;
+    for (const Unit &u : units) {
+      int begin = 0;
+      std::vector<std::pair<int, int>> where;  // (list, index in list)
+      while (begin < u.pages) {
+        if (fill >= target && c < lists - 1) {
+          ++c;
+          fill = 0;
+        }
+        const int take = (int)std::min<long long>(u.pages - begin,
+                                                  c < lists - 1 ? target - fill : u.pages - begin);
+        where.push_back({c, (int)per[c].size()});
+        per[c].push_back(WorkItem{u.b, u.j, begin, begin + take, -1, u.L, u.qpos, 0});
+        begin += take;
+        fill += take;
+      }
+      if (where.size() > 1) {
+        comb.push_back(CombineItem{u.b, u.j, slots, (int)where.size()});
+        for (size_t p = 0; p < where.size(); ++p)
+          per[where[p].first][where[p].second].slot = slots + (int)p;
+        slots += (int)where.size();
+      }
+    }
+  }
+  size_t n_items = 0;
+  for (auto &v : per) n_items += v.size();
+  if (n_items > (size_t)batch * q_len + num_ctas)
+    return fail(MLA_ERR_INVALID_ARGUMENT, "planner produced %zu items (bound %zu)", n_items,
+                (size_t)batch * q_len + num_ctas);
+  const int lists = batch == 0 ? 0 : (int)per.size();
+  unsigned char *base = static_cast<unsigned char *>(plan);
+  memset(base, 0, need);
+  PlanHeader *h = reinterpret_cast<PlanHeader *>(base);
+  h->magic = kPlanMagic;
+  h->version = kPlanVersion;
+  h->batch = batch;
+  h->q_len = q_len;
+  h->n_h = n_h;
+  h->num_items = (int)n_items;
+  h->num_ctas = lists;
+  h->num_partials = slots;
+  h->num_combine = (int)comb.size();
+  h->cta_off = (int)sizeof(PlanHeader);
+  h->items_off = h->cta_off + (int)align16(sizeof(int32_t) * (num_ctas + 1));
+  h->combine_off = h->items_off + (int)((size_t)(batch * q_len + num_ctas) * sizeof(WorkItem));
+  h->max_pages_used = max_pages_used;
+  int32_t *cta_begin = reinterpret_cast<int32_t *>(base + h->cta_off);
+  WorkItem *out_items = reinterpret_cast<WorkItem *>(base + h->items_off);
+  int n = 0;
+  for (int c = 0; c < lists; ++c) {
+    cta_begin[c] = n;
+    for (const WorkItem &it : per[c]) out_items[n++] = it;
+  }
+  cta_begin[lists] = n;
+  CombineItem *out_comb = reinterpret_cast<CombineItem *>(base + h->combine_off);
+  for (size_t i = 0; i < comb.size(); ++i) out_comb[i] = comb[i];
+  if (info) {
+    info->num_items = h->num_items;
+    info->num_ctas = h->num_ctas;
+    info->num_partials = slots;
+    info->num_combine = h->num_combine;
+    info->plan_bytes = (size_t)h->combine_off + comb.size() * sizeof(CombineItem);
+    info->workspace_bytes = workspace_bytes(slots, n_h);
+  }
+  return MLA_OK;
+}
+
+mla_status_t mla_decode_attention(const mla_bf16_t *q_full, const mla_bf16_t *cache,
+                                  int num_pages, const int32_t *block_table, int max_pages,
+                                  int batch, int q_len, int n_h, float scale,
+                                  const void *plan_host, const void *plan_dev, void *workspace,
+                                  size_t workspace_bytes_given, mla_bf16_t *o_latent, float *lse,
+                                  uint32_t *status, mla_stream_t stream) {
+  clear_error();
+  MLA_CHECK_ARG(plan_host != nullptr && plan_dev != nullptr, "plan pointers are NULL");
+  const PlanHeader *ph = static_cast<const PlanHeader *>(plan_host);
+  MLA_CHECK_ARG(ph->magic == kPlanMagic && ph->version == kPlanVersion, "not a decode plan");
+  MLA_CHECK_ARG(ph->batch == batch && ph->q_len == q_len && ph->n_h == n_h,
+                "plan was built for batch %d, q_len %d, n_h %d", ph->batch, ph->q_len, ph->n_h);
+  if (batch == 0 || ph->num_items == 0) return MLA_OK;
+  MLA_CHECK_ARG(q_full && cache && block_table && o_latent, "NULL device pointer");
+  MLA_CHECK_ARG(aligned16(q_full) && aligned16(cache) && aligned16(o_latent) &&
+                    aligned16(plan_dev) && (workspace == nullptr || aligned16(workspace)),
+                "pointers must be 16-byte aligned");
+  MLA_CHECK_ARG(num_pages > 0 && max_pages > 0, "num_pages and max_pages must be positive");
+  MLA_CHECK_ARG(ph->max_pages_used <= max_pages,
+                "a sequence needs %d pages but the block table has %d columns",
+                ph->max_pages_used, max_pages);
+  MLA_CHECK_ARG(isfinite(scale), "scale must be finite");
+  const size_t ws_need = workspace_bytes(ph->num_partials, n_h);
+  if (ph->num_partials > 0 && (workspace == nullptr || workspace_bytes_given < ws_need))
+    return fail(MLA_ERR_WORKSPACE_TOO_SMALL, "workspace %zu B < %zu B", workspace_bytes_given,
+                ws_need);
+  mla_status_t st = require_sm100();
+  if (st != MLA_OK) return st;
+  DecodeArgs a;
+  a.q_full = q_full;
+  a.cache = cache;
+  a.num_pages = num_pages;
+  a.block_table = block_table;
+  a.max_pages = max_pages;
+  a.batch = batch;
+  a.q_len = q_len;
+  a.n_h = n_h;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.plan_host = ph;
+  a.plan_dev = static_cast<const unsigned char *>(plan_dev);
+  a.ws_o = static_cast<float *>(workspace);
+  a.ws_lse = workspace ? reinterpret_cast<float *>(static_cast<unsigned char *>(workspace) +
+                                                   workspace_o_bytes(ph->num_partials, n_h))
+                       : nullptr;
+  a.o_latent = o_latent;
+  a.lse = lse;
+  a.status = status;
+  st = launch_decode(a, (cudaStream_t)stream);
+  if (st != MLA_OK) return st;
+  return launch_combine(a, (cudaStream_t)stream);
+}
+
+mla_status_t mla_out_absorb(const mla_bf16_t *o_latent, const mla_bf16_t *w_uv, int T, int n_h,
+                            mla_bf16_t *u, int ld_u, mla_stream_t stream) {
+  clear_error();
+  MLA_CHECK_ARG(T >= 0, "T < 0");
+  if (T == 0) return MLA_OK;
+  if (!heads_supported(n_h))
+    return fail(MLA_ERR_UNSUPPORTED, "n_h = %d (supported: 16..128, multiple of 16)", n_h);
+  MLA_CHECK_ARG(o_latent && w_uv && u, "NULL device pointer");
+  MLA_CHECK_ARG(aligned16(o_latent) && aligned16(w_uv) && aligned16(u),
+                "pointers must be 16-byte aligned");
+  MLA_CHECK_ARG(ld_u >= n_h * MLA_D_V && ld_u % 8 == 0, "ld_u too small or unaligned");
+  mla_status_t st = require_sm100();
+  if (st != MLA_OK) return st;
+  return launch_out_absorb(o_latent, w_uv, T, n_h, u, ld_u, (cudaStream_t)stream);
+}
+
+mla_status_t mla_gemm_bf16(const mla_bf16_t *X, int ld_x, const mla_bf16_t *W, int ld_w, void *C,
+                           int ld_c, int c_fp32, int M, int N, int K, mla_stream_t stream) {
+  clear_error();
+  MLA_CHECK_ARG(M >= 0 && N >= 0 && K >= 0, "negative size");
+  if (M == 0 || N == 0) return MLA_OK;
+  MLA_CHECK_ARG(X && W && C, "NULL device pointer");
+  MLA_CHECK_ARG(K > 0, "K must be positive");
+  MLA_CHECK_ARG(ld_x >= K && ld_w >= K && ld_c >= N, "leading dimension smaller than the row");
+  MLA_CHECK_ARG(aligned16(X) && aligned16(W) && aligned16(C), "pointers must be 16-byte aligned");
+  MLA_CHECK_ARG(ld_x % 8 == 0 && ld_w % 8 == 0 && ld_c % (c_fp32 ? 4 : 8) == 0,
+                "leading dimensions must keep rows 16-byte aligned");
+  mla_status_t st = require_sm100();
+  if (st != MLA_OK) return st;
+  return launch_projection(X, ld_x, W, ld_w, C, ld_c, c_fp32, M, N, K, (cudaStream_t)stream);
+}
+
+mla_status_t mla_read_status(uint32_t *status, uint32_t *bits, int clear, mla_stream_t stream) {
+  clear_error();
+  MLA_CHECK_ARG(status != nullptr && bits != nullptr, "NULL pointer");
+  cudaStream_t s = (cudaStream_t)stream;
+  uint32_t v = 0;
+  MLA_CUDA_TRY(cudaMemcpyAsync(&v, status, sizeof(v), cudaMemcpyDeviceToHost, s));
+  MLA_CUDA_TRY(cudaStreamSynchronize(s));
+  if (clear) {
+    MLA_CUDA_TRY(cudaMemsetAsync(status, 0, sizeof(uint32_t), s));
+    MLA_CUDA_TRY(cudaStreamSynchronize(s));
+  }
+  *bits = v;
+  if (v != 0) return fail(MLA_ERR_DEVICE, "device status bits 0x%x", v);
+  return MLA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,64 @@
+// Internal launchers shared between the translation units of the library.
+#pragma once
+
+#include "common.cuh"
+#include "plan.h"
+
+namespace mla {
+
+// Generic strided, batched bf16 GEMM on CUDA cores (fp32 accumulation):
+//   C[z][m][n] = sum_k A[z][m][k] * B[z][n][k]
+// element (z,m,k) of A at A + z*sAz + m*sAm + k*sAk, likewise B and C.
+struct GemmArgs {
+  const uint16_t *A;
+  long long sAz, sAm, sAk;
+  const uint16_t *B;
+  long long sBz, sBn, sBk;
+  void *C;
+  long long sCz, sCm, sCn;
+  int c_fp32;
+  int M, N, K, batch;
+};
+mla_status_t launch_gemm_simt(const GemmArgs &g, cudaStream_t stream);
+
+// q_full[t][h][512:576] = RoPE(q_pe[t][h][:], pos[t]) (or copy when pos == NULL).
+mla_status_t launch_q_rope_pack(const uint16_t *q_pe, int ld_qp, const int32_t *pos,
+                                const float *rope_table, int max_pos, int T, int n_h,
+                                uint16_t *q_full, uint32_t *status, cudaStream_t stream);
+
+mla_status_t launch_cache_append(uint16_t *cache, int num_pages, const int32_t *block_table,
+                                 int batch, int max_pages, const int32_t *seq_idx,
+                                 const int32_t *pos, const uint16_t *c_kv, int ld_c,
+                                 const uint16_t *k_pe, int ld_k, const float *rope_table,
+                                 int max_pos, int n_tokens, uint32_t *status,
+                                 cudaStream_t stream);
+
+struct DecodeArgs {
+  const uint16_t *q_full;
+  const uint16_t *cache;
+  int num_pages;
+  const int32_t *block_table;
+  int max_pages;
+  int batch, q_len, n_h;
+  float scale_log2;  // scale * log2(e)
+  const PlanHeader *plan_host;
+  const unsigned char *plan_dev;
+  float *ws_o;       // [num_partials][n_h][512]
+  float *ws_lse;     // [num_partials][n_h]
+  uint16_t *o_latent;
+  float *lse;
+  uint32_t *status;
+};
+mla_status_t launch_decode_simt(const DecodeArgs &a, cudaStream_t stream);
+mla_status_t launch_combine(const DecodeArgs &a, cudaStream_t stream);
+
+// The kernels behind each entry point (ops.cu).
+mla_status_t launch_absorb_q(const uint16_t *q_nope, int ld_qn, const uint16_t *w_uk, int T,
+                             int n_h, uint16_t *q_full, cudaStream_t stream);
+mla_status_t launch_out_absorb(const uint16_t *o_latent, const uint16_t *w_uv, int T, int n_h,
+                               uint16_t *u, int ld_u, cudaStream_t stream);
+mla_status_t launch_projection(const uint16_t *X, int ld_x, const uint16_t *W, int ld_w, void *C,
+                               int ld_c, int c_fp32, int M, int N, int K, cudaStream_t stream);
+mla_status_t launch_decode(const DecodeArgs &a, cudaStream_t stream);
+
+}  // namespace mla

@@ -1,0 +1,221 @@
+"""Device-resident MLA decode workloads driven through the C ABI.
+
+A session uploads one workload's tensors to the GPU (PyTorch allocates the
+memory), builds the split-KV plan, and runs decode steps as a fixed sequence
+of C-ABI calls on one CUDA stream. PyTorch is used for allocation, copies and
+streams only; every arithmetic step runs in libmla's kernels.
+"""
+
+from __future__ import annotations
+
+import math
+from typing import Optional
+
+import numpy as np
+import torch
+
+from . import mla
+
+D_C, D_R, D_NOPE, D_V, ROW, PAGE = mla.D_C, mla.D_R, mla.D_NOPE, mla.D_V, mla.ROW, mla.PAGE
+DEFAULT_SCALE = 1.0 / math.sqrt(D_NOPE + D_R)
+
+
+def to_dev_bf16(bits: np.ndarray, device) -> torch.Tensor:
+    """uint16 bf16 bit patterns -> device torch.bfloat16 tensor (same bits)."""
+    t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16))
+    return t.to(device).view(torch.bfloat16)
+
+
+def bf16_to_numpy_bits(t: torch.Tensor) -> np.ndarray:
+    return t.detach().contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def to_dev(arr: np.ndarray, device) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(arr)).to(device)
+
+
+class DecodeSession:
+    """One attention-only decode step per call of ``step()``:
+
+        mla_cache_append (RoPE on the new keys, paged scatter)
+        mla_absorb_q     (q~ = q^C W^UK, RoPE on q^R, pack [q~ | q^R])
+        mla_decode_attention (split-KV attention + combine)
+        mla_out_absorb   (u = W^UV o)
+    """
+
+    def __init__(self, inp, device="cuda", num_ctas: int = 0, max_split: int = 0,
+                 scale: float = DEFAULT_SCALE, rope_table: Optional[np.ndarray] = None):
+        w = inp.w
+        self.w = w
+        self.device = torch.device(device)
+        self.B, self.q_len, self.n_h = w.B, w.q_len, w.n_h
+        self.T = w.B * w.q_len
+        self.scale = scale
+        dev = self.device
+        self.lens = inp.lens
+        self.num_pages = inp.pool.shape[0]
+        self.max_pages = inp.table.shape[1]
+        self.cache = to_dev_bf16(inp.pool, dev)
+        self.table = to_dev(inp.table, dev)
+        self.q_nope = to_dev_bf16(inp.q_nope.reshape(self.T, -1), dev)
+        self.q_pe = to_dev_bf16(inp.q_pe.reshape(self.T, -1), dev)
+        self.c_new = to_dev_bf16(inp.c_new.reshape(self.T, D_C), dev)
+        self.k_new = to_dev_bf16(inp.k_new.reshape(self.T, D_R), dev)
+        self.w_uk = to_dev_bf16(inp.w_uk, dev)
+        self.w_uv = to_dev_bf16(inp.w_uv, dev)
+        pos = inp.positions.reshape(-1).astype(np.int32)
+        self.seq_idx = to_dev(np.repeat(np.arange(self.B, dtype=np.int32), self.q_len), dev)
+        self.pos = to_dev(pos, dev)
+        self.max_pos = int(inp.lens.max()) if rope_table is None else rope_table.shape[0]
+        tab = mla.mla_rope_table(self.max_pos) if rope_table is None else rope_table
+        self.rope = to_dev(tab, dev)
+        self.plan_host, self.info = mla.mla_decode_plan(inp.lens, self.B, self.q_len, self.n_h,
+                                                        num_ctas, max_split)
+        self.plan_dev = to_dev(self.plan_host, dev)
+        self.ws_bytes = int(self.info.workspace_bytes)
+        self.workspace = torch.empty(max(self.ws_bytes, 256), dtype=torch.uint8, device=dev)
+        self.q_full = torch.empty((self.T, self.n_h, ROW), dtype=torch.bfloat16, device=dev)
+        self.o = torch.empty((self.T, self.n_h, D_C), dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty((self.T, self.n_h), dtype=torch.float32, device=dev)
+        self.u = torch.empty((self.T, self.n_h * D_V), dtype=torch.bfloat16, device=dev)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    # the four calls of one step ------------------------------------------
+    def append(self, stream=None):
+        mla.mla_cache_append(self.cache, self.num_pages, self.table, self.B, self.max_pages,
+                             self.seq_idx, self.pos, self.c_new, D_C, self.k_new, D_R, self.rope,
+                             self.max_pos, self.T, self.status, stream)
+
+    def absorb(self, stream=None):
+        mla.mla_absorb_q(self.q_nope, self.n_h * D_NOPE, self.q_pe, self.n_h * D_R, self.w_uk,
+                         self.pos, self.rope, self.max_pos, self.T, self.n_h, self.q_full,
+                         self.status, stream)
+
+    def attend(self, stream=None, lse=True):
+        mla.mla_decode_attention(self.q_full, self.cache, self.num_pages, self.table,
+                                 self.max_pages, self.B, self.q_len, self.n_h, self.scale,
+                                 self.plan_host, self.plan_dev, self.workspace, self.ws_bytes,
+                                 self.o, self.lse if lse else None, self.status, stream)
+
+    def expand(self, stream=None):
+        mla.mla_out_absorb(self.o, self.w_uv, self.T, self.n_h, self.u, self.n_h * D_V, stream)
+
+    def step(self, stream=None):
+        self.append(stream)
+        self.absorb(stream)
+        self.attend(stream)
+        self.expand(stream)
+
+    def read_status(self) -> int:
+        return mla.mla_read_status(self.status, clear=True)
+
+    # e2e: per-step inputs from pinned host memory, result back to host ----
+    def pinned_step_buffers(self):
+        """Pinned host copies of the per-step inputs and of the result."""
+        ins = [self.q_nope, self.q_pe, self.c_new, self.k_new]
+        host_in = [t.cpu().pin_memory() for t in ins]
+        host_out = torch.empty(self.u.shape, dtype=self.u.dtype).pin_memory()
+        return ins, host_in, host_out
+
+    def step_e2e(self, ins, host_in, host_out, stream=None):
+        for d, h in zip(ins, host_in):
+            d.copy_(h, non_blocking=True)
+        self.step(stream)
+        host_out.copy_(self.u, non_blocking=True)
+
+    @staticmethod
+    def step_io_bytes(ins, host_out) -> tuple:
+        return (sum(t.numel() * t.element_size() for t in ins),
+                host_out.numel() * host_out.element_size())
+
+
+class LayerSession:
+    """A whole MLA decode layer from hidden states:
+
+        [c^Q =] h W_DQ^T ; [q^C | q^R] = (c^Q or h) [W_UQ|W_QR]^T   (mla_gemm_bf16)
+        [c^KV | k^R] = h [W_DKV|W_KR]^T                              (mla_gemm_bf16)
+        mla_cache_append, mla_absorb_q, mla_decode_attention, mla_out_absorb
+        out = u W_O^T (float32)                                      (mla_gemm_bf16)
+
+    The rows of h that are queries must be the last B*q_len rows.
+    """
+
+    def __init__(self, inp, device="cuda", num_ctas: int = 0, max_split: int = 0,
+                 scale: float = DEFAULT_SCALE):
+        w = inp.w
+        self.w = w
+        dev = self.device = torch.device(device)
+        self.B, self.q_len, self.n_h = w.B, w.q_len, w.n_h
+        self.Tq = w.B * w.q_len
+        self.T = inp.h.shape[0]
+        assert np.array_equal(inp.query_tok, np.arange(self.T - self.Tq, self.T))
+        self.scale = scale
+        self.hidden = w.hidden
+        self.q_lora = w.q_lora
+        W = inp.weights
+        self.lens = inp.lens
+        self.num_pages = inp.pool.shape[0]
+        self.max_pages = inp.table.shape[1]
+        self.cache = to_dev_bf16(inp.pool, dev)
+        self.table = to_dev(inp.table, dev)
+        self.h = to_dev_bf16(inp.h, dev)
+        if self.q_lora:
+            self.w_dq = to_dev_bf16(W["w_dq"], dev)
+            self.w_qcat = to_dev_bf16(np.concatenate([W["w_uq"], W["w_qr"]], 0), dev)
+        else:
+            self.w_qcat = to_dev_bf16(np.concatenate([W["w_q"], W["w_qr"]], 0), dev)
+        self.w_kvcat = to_dev_bf16(np.concatenate([W["w_dkv"], W["w_kr"]], 0), dev)
+        self.w_uk = to_dev_bf16(W["w_uk"], dev)
+        self.w_uv = to_dev_bf16(W["w_uv"], dev)
+        self.w_o = to_dev_bf16(W["w_o"], dev)
+        self.tok_seq = to_dev(inp.tok_seq, dev)
+        self.tok_pos = to_dev(inp.tok_pos, dev)
+        self.q_pos = to_dev(inp.tok_pos[self.T - self.Tq:], dev)
+        self.max_pos = int(inp.lens.max())
+        self.rope = to_dev(mla.mla_rope_table(self.max_pos), dev)
+        self.plan_host, self.info = mla.mla_decode_plan(inp.lens, self.B, self.q_len, self.n_h,
+                                                        num_ctas, max_split)
+        self.plan_dev = to_dev(self.plan_host, dev)
+        self.ws_bytes = int(self.info.workspace_bytes)
+        self.workspace = torch.empty(max(self.ws_bytes, 256), dtype=torch.uint8, device=dev)
+        nq = self.n_h * (D_NOPE + D_R)
+        self.cq = (torch.empty((self.Tq, self.q_lora), dtype=torch.bfloat16, device=dev)
+                   if self.q_lora else None)
+        self.q = torch.empty((self.Tq, nq), dtype=torch.bfloat16, device=dev)
+        self.kv = torch.empty((self.T, ROW), dtype=torch.bfloat16, device=dev)
+        self.q_full = torch.empty((self.Tq, self.n_h, ROW), dtype=torch.bfloat16, device=dev)
+        self.o = torch.empty((self.Tq, self.n_h, D_C), dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty((self.Tq, self.n_h), dtype=torch.float32, device=dev)
+        self.u = torch.empty((self.Tq, self.n_h * D_V), dtype=torch.bfloat16, device=dev)
+        self.out = torch.empty((self.Tq, self.hidden), dtype=torch.float32, device=dev)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def step(self, stream=None):
+        n_h, d = self.n_h, self.hidden
+        hq = self.h[self.T - self.Tq:]
+        nq = n_h * (D_NOPE + D_R)
+        if self.q_lora:
+            mla.mla_gemm_bf16(hq, d, self.w_dq, d, self.cq, self.q_lora, 0, self.Tq, self.q_lora,
+                              d, stream)
+            mla.mla_gemm_bf16(self.cq, self.q_lora, self.w_qcat, self.q_lora, self.q, nq, 0,
+                              self.Tq, nq, self.q_lora, stream)
+        else:
+            mla.mla_gemm_bf16(hq, d, self.w_qcat, d, self.q, nq, 0, self.Tq, nq, d, stream)
+        mla.mla_gemm_bf16(self.h, d, self.w_kvcat, d, self.kv, ROW, 0, self.T, ROW, d, stream)
+        kv_pe = self.kv[:, D_C:]
+        mla.mla_cache_append(self.cache, self.num_pages, self.table, self.B, self.max_pages,
+                             self.tok_seq, self.tok_pos, self.kv, ROW, kv_pe, ROW, self.rope,
+                             self.max_pos, self.T, self.status, stream)
+        q_pe = self.q[:, n_h * D_NOPE:]
+        mla.mla_absorb_q(self.q, nq, q_pe, nq, self.w_uk, self.q_pos, self.rope, self.max_pos,
+                         self.Tq, n_h, self.q_full, self.status, stream)
+        mla.mla_decode_attention(self.q_full, self.cache, self.num_pages, self.table,
+                                 self.max_pages, self.B, self.q_len, n_h, self.scale,
+                                 self.plan_host, self.plan_dev, self.workspace, self.ws_bytes,
+                                 self.o, self.lse, self.status, stream)
+        mla.mla_out_absorb(self.o, self.w_uv, self.Tq, n_h, self.u, n_h * D_V, stream)
+        mla.mla_gemm_bf16(self.u, n_h * D_V, self.w_o, n_h * D_V, self.out, d, 1, self.Tq, d,
+                          n_h * D_V, stream)
+
+    def read_status(self) -> int:
+        return mla.mla_read_status(self.status, clear=True)

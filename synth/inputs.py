@@ -198,8 +198,10 @@ def attention_weights(w: Workload):
     return w_uk, w_uv
 
 
-def make_decode_inputs(w: Workload, with_pool: bool = True) -> DecodeInputs:
-    lens = seq_lens(w)
+def make_decode_inputs(w: Workload, with_pool: bool = True, lens=None) -> DecodeInputs:
+    """Inputs of workload w; ``lens`` overrides its sequence lengths."""
+    lens = seq_lens(w) if lens is None else np.asarray(lens, dtype=np.int32)
+    assert lens.shape == (w.B,) and lens.min() >= w.q_len
     table = block_table(w, lens)
     pool = build_pool(w, lens, table) if with_pool else None
     q_nope = normal_bf16(stream(w.seed, S_QNOPE), (w.B, w.q_len, w.n_h, D_NOPE))
@@ -232,9 +234,11 @@ class LayerInputs:
     weights: Dict[str, np.ndarray]
 
 
-def make_layer_inputs(w: Workload, with_pool: bool = True) -> LayerInputs:
+def make_layer_inputs(w: Workload, with_pool: bool = True, lens=None) -> LayerInputs:
+    """Inputs of layer workload w; ``lens`` overrides its sequence lengths."""
     assert w.layer
-    lens = seq_lens(w)
+    lens = seq_lens(w) if lens is None else np.asarray(lens, dtype=np.int32)
+    assert lens.shape == (w.B,) and lens.min() >= w.q_len
     table = block_table(w, lens)
     pool = build_pool(w, lens, table) if with_pool else None
     if w.synth_prefix:

@@ -1,0 +1,150 @@
+"""CPU tests of the C-ABI library: it loads, exports every declared symbol,
+validates arguments before touching the GPU, and its host planner and RoPE
+table are correct. No test here launches a kernel."""
+
+import ctypes
+import glob
+import os
+import re
+
+import numpy as np
+import pytest
+
+from mla_latent_kv_32_b200 import build as build_mod
+from mla_latent_kv_32_b200 import mla
+from oracle import mla_oracle as O
+from tests._plan import parse_plan
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build_mod.build()
+    return mla.load()
+
+
+def declared_symbols():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(h).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", "", src)
+        for m in re.finditer(r"\b(mla_[a-z0-9_]+)\s*\(", src):
+            names.add(m.group(1))
+    return sorted(names)
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_symbols()
+    assert "mla_decode_attention" in names and len(names) >= 10
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in include/ but not exported"
+    # the binding covers the same set
+    for n in names:
+        assert n in mla.SIGNATURES, f"{n} has no Python binding"
+
+
+def test_invalid_arguments_rejected_before_launch(lib):
+    with pytest.raises(mla.MlaError) as e:
+        mla.mla_cache_append(None, 1, None, 1, 1, None, None, None, 512, None, 64, None, 1, 4,
+                             stream=0)
+    assert e.value.status == mla.MLA_ERR_INVALID_ARGUMENT
+    with pytest.raises(mla.MlaError) as e:
+        mla.mla_absorb_q(16, 2048, 16, 1024, 16, None, None, 0, 1, 24, 16, stream=0)
+    assert e.value.status == mla.MLA_ERR_UNSUPPORTED
+    with pytest.raises(mla.MlaError) as e:
+        mla.mla_gemm_bf16(16, 8, 16, 8, 8, 8, 0, 4, 4, 8, stream=0)   # C misaligned
+    assert e.value.status == mla.MLA_ERR_INVALID_ARGUMENT
+    # zero-sized calls are no-ops that succeed without a device
+    mla.mla_cache_append(None, 1, None, 1, 1, None, None, None, 512, None, 64, None, 1, 0, stream=0)
+    mla.mla_out_absorb(None, None, 0, 128, None, 16384, stream=0)
+
+
+def test_rope_table_matches_oracle(lib):
+    got = mla.mla_rope_table(140000)
+    want = O.rope_table(140000)
+    # Both round a float64 cos/sin to float32. The float64 angles may differ in
+    # their last bit (the two pow implementations differ), which flips the
+    # float32 rounding when the value sits next to a rounding midpoint: the
+    # tables then differ by one float32 ulp in a handful of entries.
+    d = np.abs(got.astype(np.float64) - want.astype(np.float64))
+    assert d.max() <= 2.0 ** -24 * 1.0001
+    assert (got != want).mean() < 1e-4
+    with pytest.raises(mla.MlaError):
+        mla.mla_rope_table(0)
+
+
+def check_plan(lens, q_len, num_ctas, max_split=0, n_h=128):
+    lens = np.asarray(lens, np.int32)
+    B = len(lens)
+    buf, info = mla.mla_decode_plan(lens, B, q_len, n_h, num_ctas, max_split)
+    p = parse_plan(buf)
+    assert p["num_items"] == info.num_items and p["num_partials"] == info.num_partials
+    assert p["num_items"] <= B * q_len + num_ctas
+    cover = {}
+    for it in p["items"]:
+        key = (it["b"], it["j"])
+        L = int(lens[it["b"]])
+        assert it["L"] == L and it["qpos"] == L - q_len + it["j"]
+        assert 0 <= it["page_begin"] < it["page_end"]
+        cover.setdefault(key, []).append(it)
+    assert len(cover) == B * q_len
+    slots = set()
+    for (b, j), its in cover.items():
+        need = (int(lens[b]) - q_len + j + 1 + 63) // 64
+        rng = sorted((i["page_begin"], i["page_end"]) for i in its)
+        assert rng[0][0] == 0 and rng[-1][1] == need
+        for a, c in zip(rng, rng[1:]):
+            assert a[1] == c[0]
+        if len(its) == 1:
+            assert its[0]["slot"] == -1
+        else:
+            ss = sorted(i["slot"] for i in its)
+            assert ss == list(range(ss[0], ss[0] + len(its)))
+            slots.update(ss)
+            ci = [c for c in p["combine"] if (c["b"], c["j"]) == (b, j)]
+            assert len(ci) == 1 and ci[0]["first_slot"] == ss[0] and ci[0]["n_parts"] == len(its)
+    assert len(slots) == p["num_partials"]
+    # work lists partition the items
+    cb = p["cta_begin"]
+    assert cb[0] == 0 and cb[-1] == p["num_items"] and np.all(np.diff(cb) >= 0)
+    loads = [sum(p["items"][k]["page_end"] - p["items"][k]["page_begin"]
+                 for k in range(cb[c], cb[c + 1])) for c in range(p["num_ctas"])]
+    total = sum(need for need in
+                [(int(lens[b]) - q_len + j + 1 + 63) // 64 for b in range(B) for j in range(q_len)])
+    assert sum(loads) == total
+    return p, loads, total
+
+
+@pytest.mark.parametrize("lens,q_len,ctas", [
+    ([4096] * 64, 1, 74), ([1, 63, 64, 65, 127, 200], 1, 3), ([2, 131072, 5000, 64], 2, 74),
+    ([1], 1, 74), ([300] * 7, 2, 1)])
+def test_planner_contiguous_cuts(lens, q_len, ctas):
+    p, loads, total = check_plan(lens, q_len, ctas)
+    assert max(loads) <= -(-total // min(ctas, total))
+
+
+def test_planner_ragged_workload_balanced():
+    import synth
+    w = synth.WORKLOADS["ragged"]
+    lens = synth.seq_lens(w)
+    p, loads, total = check_plan(lens, 1, 74)
+    assert max(loads) - min(loads) <= 1 or max(loads) <= -(-total // 74)
+
+
+def test_planner_no_split_mode():
+    p, loads, total = check_plan([4096] * 64, 1, 74, max_split=1)
+    assert p["num_partials"] == 0 and p["num_items"] == 64
+    assert max(loads) == 64
+
+
+def test_planner_rejects_bad_input():
+    with pytest.raises(mla.MlaError):
+        mla.mla_decode_plan(np.array([1, 0], np.int32), 2, 1, 128, 8)    # L < q_len
+    with pytest.raises(mla.MlaError):
+        mla.mla_decode_plan(np.array([5], np.int32), 1, 3, 128, 8)       # q_len 3
+    with pytest.raises(mla.MlaError):
+        mla.mla_decode_plan(np.array([5], np.int32), 1, 1, 100, 8)       # n_h 100
+    buf, info = mla.mla_decode_plan(np.zeros(0, np.int32), 0, 1, 128, 8)
+    assert info.num_items == 0

@@ -1,0 +1,52 @@
+"""GPU parity of the whole decode layer (projections, RoPE, append, absorbed
+attention, W_UV, W_O) against the fp64 oracle's layer, through the C ABI."""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from mla_latent_kv_32_b200 import build as build_mod
+from mla_latent_kv_32_b200 import mla
+from mla_latent_kv_32_b200.runtime import LayerSession, bf16_to_numpy_bits
+from oracle import mla_oracle as O
+from tests._util import assert_parity
+
+pytestmark = pytest.mark.gpu
+SCALE = 1.0 / math.sqrt(192)
+
+
+@pytest.fixture(scope="module")
+def dev():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    build_mod.build()
+    mla.load()
+    return torch.device("cuda:0")
+
+
+@pytest.mark.parametrize("name", ["tiny", "layer_v3"])
+def test_layer(dev, name):
+    w = synth.WORKLOADS[name]
+    inp = synth.make_layer_inputs(w)
+    sess = LayerSession(inp, dev)
+    sess.step()
+    torch.cuda.synchronize()
+    assert sess.read_status() == 0
+    seqs = [0] if w.B == 1 else synth.sample_sequences(w, inp.lens, 6)
+    ref = O.layer_decode(inp.h, inp.weights, w.n_h, w.q_len, inp.tok_seq, inp.tok_pos,
+                         inp.query_tok, lambda b, n: synth.prefix_rows(w, b, n), inp.lens,
+                         SCALE, seqs)
+    rows = np.concatenate([np.arange(b * w.q_len, (b + 1) * w.q_len) for b in seqs])
+    out = sess.out.cpu().numpy()[rows]
+    u = sess.u.float().cpu().numpy()[rows].reshape(-1, w.n_h, 128)
+    assert_parity(u, ref["u"], "u")
+    assert_parity(out, ref["out"], "layer output")
+    # the rows the layer appended, against the oracle's float64 chain (tolerance:
+    # the GPU rounds the projection to bf16 before the RoPE, the oracle after)
+    pool = bf16_to_numpy_bits(sess.cache)
+    got = np.stack([pool[inp.table[inp.tok_seq[t], inp.tok_pos[t] // 64], inp.tok_pos[t] % 64]
+                    for t in ref["new_tok"]])
+    assert_parity(O.bf16_to_f64(got), O.bf16_to_f64(ref["new_rows"]), "appended rows")
