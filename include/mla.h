@@ -203,6 +203,32 @@ mla_status_t mla_decode_attention(const mla_bf16_t *q_full, const mla_bf16_t *ca
                                   mla_stream_t stream);
 
 /*
+ * mla_decode_attention_noalloc -- device. The same attention as
+ * mla_decode_attention, for callers that cannot allocate device memory at the
+ * time of the call: code being captured into a CUDA graph, a serving engine
+ * that has reserved the GPU's memory for its own cache pool, a plugin running
+ * under another framework's allocator. The pages describe no such variant;
+ * it exists only for those callers.
+ * Instead of a caller-supplied workspace, the split-KV partial results go to a
+ * fixed 48 MiB array inside the library (allocated on every GPU that loads the
+ * library, held until the process exits). The caller still passes all inputs
+ * and outputs. The first call on each device looks up the array's address
+ * (with that device current); make that first call before any stream capture.
+ * Every call shares the array and it keeps the previous call's contents;
+ * nothing in it needs to start at zero. Calls that can overlap on the GPU
+ * (other streams or host threads) race on the array: serialise them.
+ * No cudaMalloc, cudaFree or other allocating routine is called.
+ * Errors: as mla_decode_attention; WORKSPACE_TOO_SMALL when the plan needs more
+ * than 48 MiB of partial results (plan with fewer splits, e.g. max_split = 1).
+ */
+mla_status_t mla_decode_attention_noalloc(const mla_bf16_t *q_full, const mla_bf16_t *cache,
+                                          int num_pages, const int32_t *block_table,
+                                          int max_pages, int batch, int q_len, int n_h,
+                                          float scale, const void *plan_host,
+                                          const void *plan_dev, mla_bf16_t *o_latent,
+                                          float *lse, uint32_t *status, mla_stream_t stream);
+
+/*
  * mla_out_absorb -- device. Expands the latent attention output through W^UV:
  *   u[t][h*128 + d] = sum_c o_latent[t][h][c] * w_uv[h][d][c]
  * ("DeepSeek-V3 MLA ... Guide", "The Matrix Absorption Trick", part 3:
