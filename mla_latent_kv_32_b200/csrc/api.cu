@@ -11,6 +11,7 @@
 #include <vector>
 
 #include "internal.h"
+#include "mla_debug.h"
 
 namespace mla {
 
@@ -296,12 +297,16 @@ mla_status_t mla_decode_plan(const int32_t *seq_lens, int batch, int q_len, int 
   return MLA_OK;
 }
 
-mla_status_t mla_decode_attention(const mla_bf16_t *q_full, const mla_bf16_t *cache,
-                                  int num_pages, const int32_t *block_table, int max_pages,
-                                  int batch, int q_len, int n_h, float scale,
-                                  const void *plan_host, const void *plan_dev, void *workspace,
-                                  size_t workspace_bytes_given, mla_bf16_t *o_latent, float *lse,
-                                  uint32_t *status, mla_stream_t stream) {
+}  // extern "C"
+
+// Validation and launch shared by the decode entry points; `cuda_cores`
+// selects the CUDA-core kernel (debug entry point) instead of the tensor-core one.
+static mla_status_t decode_entry(const mla_bf16_t *q_full, const mla_bf16_t *cache,
+                                 int num_pages, const int32_t *block_table, int max_pages,
+                                 int batch, int q_len, int n_h, float scale,
+                                 const void *plan_host, const void *plan_dev, void *workspace,
+                                 size_t workspace_bytes_given, mla_bf16_t *o_latent, float *lse,
+                                 uint32_t *status, mla_stream_t stream, bool cuda_cores) {
   clear_error();
   MLA_CHECK_ARG(plan_host != nullptr && plan_dev != nullptr, "plan pointers are NULL");
   const PlanHeader *ph = static_cast<const PlanHeader *>(plan_host);
@@ -343,9 +348,35 @@ mla_status_t mla_decode_attention(const mla_bf16_t *q_full, const mla_bf16_t *ca
   a.o_latent = o_latent;
   a.lse = lse;
   a.status = status;
-  st = launch_decode(a, (cudaStream_t)stream);
+  st = cuda_cores ? launch_decode_simt(a, (cudaStream_t)stream)
+                  : launch_decode(a, (cudaStream_t)stream);
   if (st != MLA_OK) return st;
   return launch_combine(a, (cudaStream_t)stream);
+}
+
+extern "C" {
+
+mla_status_t mla_decode_attention(const mla_bf16_t *q_full, const mla_bf16_t *cache,
+                                  int num_pages, const int32_t *block_table, int max_pages,
+                                  int batch, int q_len, int n_h, float scale,
+                                  const void *plan_host, const void *plan_dev, void *workspace,
+                                  size_t workspace_bytes_given, mla_bf16_t *o_latent, float *lse,
+                                  uint32_t *status, mla_stream_t stream) {
+  return decode_entry(q_full, cache, num_pages, block_table, max_pages, batch, q_len, n_h, scale,
+                      plan_host, plan_dev, workspace, workspace_bytes_given, o_latent, lse,
+                      status, stream, false);
+}
+
+mla_status_t mla_decode_attention_cudacore(const mla_bf16_t *q_full, const mla_bf16_t *cache,
+                                           int num_pages, const int32_t *block_table,
+                                           int max_pages, int batch, int q_len, int n_h,
+                                           float scale, const void *plan_host,
+                                           const void *plan_dev, void *workspace,
+                                           size_t workspace_bytes_given, mla_bf16_t *o_latent,
+                                           float *lse, uint32_t *status, mla_stream_t stream) {
+  return decode_entry(q_full, cache, num_pages, block_table, max_pages, batch, q_len, n_h, scale,
+                      plan_host, plan_dev, workspace, workspace_bytes_given, o_latent, lse,
+                      status, stream, true);
 }
 
 mla_status_t mla_out_absorb(const mla_bf16_t *o_latent, const mla_bf16_t *w_uv, int T, int n_h,

@@ -62,6 +62,8 @@ SIGNATURES = {
     "mla_decode_plan": (_I, [_P, _I, _I, _I, _I, _I, _P, _SZ, ctypes.POINTER(mla_plan_info_t)]),
     "mla_decode_attention": (_I, [_P, _P, _I, _P, _I, _I, _I, _I, _F, _P, _P, _P, _SZ, _P, _P,
                                   _P, _P]),
+    "mla_decode_attention_cudacore": (_I, [_P, _P, _I, _P, _I, _I, _I, _I, _F, _P, _P, _P, _SZ,
+                                           _P, _P, _P, _P]),
     "mla_decode_attention_noalloc": (_I, [_P, _P, _I, _P, _I, _I, _I, _I, _F, _P, _P, _P, _P,
                                           _P, _P]),
     "mla_out_absorb": (_I, [_P, _P, _I, _I, _P, _I, _P]),
@@ -163,6 +165,18 @@ def mla_decode_attention(q_full, cache, num_pages, block_table, max_pages, batch
                                        _ptr(plan_dev), _ptr(workspace), workspace_bytes,
                                        _ptr(o_latent), _ptr(lse), _ptr(status),
                                        _stream(stream)), "mla_decode_attention")
+
+
+def mla_decode_attention_cudacore(q_full, cache, num_pages, block_table, max_pages, batch, q_len,
+                                  n_h, scale, plan_host, plan_dev, workspace, workspace_bytes,
+                                  o_latent, lse=None, status=None, stream=None):
+    """Debug entry point: the same attention on CUDA cores (differential tests)."""
+    _check(load().mla_decode_attention_cudacore(_ptr(q_full), _ptr(cache), num_pages,
+                                                _ptr(block_table), max_pages, batch, q_len, n_h,
+                                                scale, _ptr(plan_host), _ptr(plan_dev),
+                                                _ptr(workspace), workspace_bytes, _ptr(o_latent),
+                                                _ptr(lse), _ptr(status), _stream(stream)),
+           "mla_decode_attention_cudacore")
 
 
 def mla_decode_attention_noalloc(q_full, cache, num_pages, block_table, max_pages, batch, q_len,

@@ -165,3 +165,28 @@ def test_workload_full_size(dev, name):
             p = int(pos[b, j])
             want = O.make_cache_row(inp.c_new[b, j], inp.k_new[b, j], [p], table)[0]
             assert np.array_equal(pool[inp.table[b, p // 64], p % 64], want)
+
+
+@pytest.mark.parametrize("lens,q_len,n_h,ctas", [
+    ([700, 64, 1, 129, 2000], 1, 128, 74), ([300, 4100], 2, 128, 16), ([90, 33], 1, 48, 3)])
+def test_tensor_core_vs_cuda_core(dev, lens, q_len, n_h, ctas):
+    """Two independent GPU kernels on the same inputs and plan agree."""
+    w = synth.Workload("diff", B=len(lens), q_len=q_len, L=max(lens), n_h=n_h, seed=13)
+    inp = synth.make_decode_inputs(w, lens=[max(l, q_len) for l in lens])
+    sess = DecodeSession(inp, dev, num_ctas=ctas)
+    sess.append()
+    sess.absorb()
+    sess.attend()
+    torch.cuda.synchronize()
+    o_tc = sess.o.float().cpu().numpy()
+    lse_tc = sess.lse.cpu().numpy()
+    o_cc = torch.empty_like(sess.o)
+    lse_cc = torch.empty_like(sess.lse)
+    mla.mla_decode_attention_cudacore(sess.q_full, sess.cache, sess.num_pages, sess.table,
+                                      sess.max_pages, sess.B, sess.q_len, sess.n_h, sess.scale,
+                                      sess.plan_host, sess.plan_dev, sess.workspace, sess.ws_bytes,
+                                      o_cc, lse_cc, sess.status)
+    torch.cuda.synchronize()
+    assert sess.read_status() == 0
+    assert_parity(o_tc, o_cc.float().cpu().numpy(), "o: tensor-core vs CUDA-core kernel")
+    assert np.max(np.abs(lse_tc - lse_cc.cpu().numpy())) <= 1e-2
