@@ -402,6 +402,7 @@ mla_status_t mla_gemm_bf16(const mla_bf16_t *X, int ld_x, const mla_bf16_t *W, i
   if (M == 0 || N == 0) return MLA_OK;
   MLA_CHECK_ARG(X && W && C, "NULL device pointer");
   MLA_CHECK_ARG(K > 0, "K must be positive");
+  if (K % 16 != 0) return fail(MLA_ERR_UNSUPPORTED, "K = %d (must be a multiple of 16)", K);
   MLA_CHECK_ARG(ld_x >= K && ld_w >= K && ld_c >= N, "leading dimension smaller than the row");
   MLA_CHECK_ARG(aligned16(X) && aligned16(W) && aligned16(C), "pointers must be 16-byte aligned");
   MLA_CHECK_ARG(ld_x % 8 == 0 && ld_w % 8 == 0 && ld_c % (c_fp32 ? 4 : 8) == 0,

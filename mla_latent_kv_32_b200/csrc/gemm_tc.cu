@@ -1,0 +1,254 @@
+// Batched bf16 GEMM on the sm_100a tensor cores (tcgen05, TMA, TMEM), fp32
+// accumulation, for the absorbed-MLA contractions around the attention:
+//   W^UK folded into the query:   q~[t][h][c] = sum_d q^C[t][h][d] W^UK[h][d][c]
+//   W^UV applied to the output:   u[t][h][d]  = sum_c o[t][h][c]  W^UV[h][d][c]
+//   and the decode layer's projections (W^DQ, [W^UQ|W^QR], [W^DKV|W^KR], W^O)
+// ("DeepSeek-V3 MLA: Multi-Head Latent Attention Guide", "The Matrix
+// Absorption Trick" parts 2-3, "Core Architecture & Mathematics" 1-2).
+//
+// Every use has few tokens and a large weight, so the weight is the M side
+// (tiles of 128 rows, the tensor core's native height) and the tokens are the
+// N side (16..256 per tile):
+//   C[z][m][n] = sum_k A[z][m][k] * B[z][n][k]
+// A (the weight) is K-major or MN-major in global memory, B (the activations)
+// is K-major; both arrive through 3-D TMA tensor maps (z = head or split) in
+// 64-element k-chunks with the 128-byte swizzle. One CTA computes one
+// 128 x BN tile: warp 0 lane 0 issues TMA into a 4-stage ring, warp 1 lane 0
+// issues the MMAs into a TMEM accumulator, all four warps then read it back
+// (thread = row m) and write C through arbitrary strides, as bf16 or fp32
+// (fp32 outputs may be split over K and reduced with atomic adds).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace mla {
+namespace {
+
+using namespace sm100;
+
+constexpr int kStages = 4;
+constexpr uint32_t kAStage = 128 * 128;        // 128 rows x 64 k (bf16) = 16 KB
+constexpr uint32_t kBStageMax = 256 * 128;     // up to 256 rows x 64 k = 32 KB
+constexpr uint32_t kStageBytes = kAStage + kBStageMax;
+constexpr uint32_t kOffBar = kStages * kStageBytes;  // 196608
+constexpr uint32_t kSmemBytes = kOffBar + 128 + 1024;
+constexpr uint64_t kTimeoutNs = 1000000000ull;
+
+struct GemmTcArgs {
+  int M, N, K;          // per batch
+  int BN;               // tile width in n (multiple of 16, <= 256)
+  int k_chunks;         // 64-element k-chunks per split
+  int splits;           // split-K factor (fp32 output only)
+  int batch;
+  int a_mn;             // A is MN-major (m contiguous)
+  void *C;
+  long long sCz, sCm, sCn;
+  int c_fp32;
+  uint32_t *status;
+};
+
+__device__ __noinline__ bool wait_bar_g(uint32_t bar, uint32_t parity, uint32_t *status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63) == 0 && globaltimer_ns() - t0 > kTimeoutNs) {
+      report(status, MLA_DEV_TIMEOUT);
+      return false;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(128, 1)
+gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+               const GemmTcArgs g) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  unsigned char *smem = smem_raw + (base - raw);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n0 = blockIdx.x * g.BN;
+  const int m0 = blockIdx.y * 128;
+  const int z = blockIdx.z / g.splits;
+  const int split = blockIdx.z % g.splits;
+  const int kc0 = split * g.k_chunks;
+  const int kc1 = min(kc0 + g.k_chunks, (g.K + 63) / 64);
+  const uint32_t bar_full = base + kOffBar, bar_empty = bar_full + 8 * kStages;
+  const uint32_t bar_done = bar_empty + 8 * kStages, tptr = bar_done + 8;
+  const uint32_t b_bytes = (uint32_t)g.BN * 128;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(bar_full + 8 * i, 1);
+      mbar_init(bar_empty + 8 * i, 1);
+    }
+    mbar_init(bar_done, 1);
+    fence_mbar_init_cluster();
+  }
+  if (warp == 1) tmem_alloc(tptr, 256);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + (tptr - base));
+
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_a);
+    tma_prefetch_desc(&tm_b);
+    int armed[kStages] = {};
+    for (int kc = kc0, i = 0; kc < kc1; ++kc, ++i) {
+      const int s = i % kStages;
+      if (i >= kStages && !wait_bar_g(bar_empty + 8 * s, ((i / kStages) - 1) & 1, g.status))
+        break;
+      const uint32_t a_s = base + s * kStageBytes, b_s = a_s + kAStage;
+      mbar_arrive_expect_tx(bar_full + 8 * s, kAStage + b_bytes);
+      ++armed[s];
+      if (g.a_mn) {
+        // two 64-row (m) boxes of 64 k-rows each
+        tma_load_3d(a_s, &tm_a, m0, kc * 64, z, bar_full + 8 * s);
+        tma_load_3d(a_s + 8192, &tm_a, m0 + 64, kc * 64, z, bar_full + 8 * s);
+      } else {
+        tma_load_3d(a_s, &tm_a, kc * 64, m0, z, bar_full + 8 * s);
+      }
+      tma_load_3d(b_s, &tm_b, kc * 64, n0, z, bar_full + 8 * s);
+    }
+    for (int s = 0; s < kStages; ++s)
+      if (armed[s]) wait_bar_g(bar_full + 8 * s, (armed[s] - 1) & 1, g.status);
+  } else if (warp == 1 && lane == 0) {
+    const uint32_t idesc = idesc_bf16(128, g.BN, g.a_mn, 0);
+    for (int kc = kc0, i = 0; kc < kc1; ++kc, ++i) {
+      const int s = i % kStages;
+      if (!wait_bar_g(bar_full + 8 * s, (i / kStages) & 1, g.status)) break;
+      tc_fence_after();
+      const uint32_t a_s = base + s * kStageBytes, b_s = a_s + kAStage;
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint64_t ad = g.a_mn ? smem_desc(a_s + kk * 2048, 8192, 1024, kSwizzle128B)
+                                   : smem_desc(a_s + kk * 32, 16, 1024, kSwizzle128B);
+        const uint64_t bd = smem_desc(b_s + kk * 32, 16, 1024, kSwizzle128B);
+        mma_f16_ss(tmem, ad, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+      }
+      mma_commit(bar_empty + 8 * s);
+    }
+    mma_commit(bar_done);
+  }
+  __syncwarp();
+  // epilogue: thread = row m of the tile
+  const bool done = wait_bar_g(bar_done, 0, g.status);
+  tc_fence_after();
+  const int m = m0 + threadIdx.x;
+  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  for (int ch = 0; ch * 32 < g.BN; ++ch) {
+    uint32_t r[32];
+    tmem_ld32(tmem + lane_off + 32 * ch, r);
+    tmem_wait_ld();
+    if (!done || kc1 <= kc0 || m >= g.M) continue;
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      const int n = n0 + 32 * ch + e;
+      if (n >= g.N) break;
+      const long long off = (long long)z * g.sCz + (long long)m * g.sCm + (long long)n * g.sCn;
+      const float v = __uint_as_float(r[e]);
+      if (g.c_fp32) {
+        if (g.splits > 1)
+          atomicAdd(reinterpret_cast<float *>(g.C) + off, v);
+        else
+          reinterpret_cast<float *>(g.C)[off] = v;
+      } else {
+        reinterpret_cast<uint16_t *>(g.C)[off] = (uint16_t)f32_to_bf16_bits(v);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 3-D bf16 tensor: dim0 contiguous (d0 elements), dim1 stride s1 elements,
+// dim2 stride s2 elements; box {64, box1, 1} with the 128-byte swizzle.
+mla_status_t make_map3(CUtensorMap *tm, const void *ptr, uint64_t d0, uint64_t d1, uint64_t d2,
+                       uint64_t s1, uint64_t s2, uint32_t box1) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = encoder();
+  if (enc == nullptr) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  if (((s1 * 2) & 15) || ((s2 * 2) & 15))
+    return fail(MLA_ERR_INVALID_ARGUMENT, "GEMM operand strides must be multiples of 16 bytes");
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {s1 * 2, s2 * 2};
+  cuuint32_t box[3] = {64, box1, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return MLA_OK;
+}
+
+}  // namespace
+
+mla_status_t launch_gemm_tc(const GemmTcDesc &d, cudaStream_t stream) {
+  if (d.M == 0 || d.N == 0 || d.batch == 0) return MLA_OK;
+  if (d.K <= 0 || d.K % 16 != 0) return fail(MLA_ERR_UNSUPPORTED, "GEMM K must be a multiple of 16");
+  CUtensorMap tm_a, tm_b;
+  const int BN = d.N >= 256 ? 256 : ((d.N + 15) / 16) * 16;
+  mla_status_t st;
+  if (d.a_mn)  // A element (z, m, k) at A + z*sAz + k*sAk + m (m contiguous)
+    st = make_map3(&tm_a, d.A, d.M, d.K, d.batch, d.sAk, d.sAz, 64);
+  else         // A element (z, m, k) at A + z*sAz + m*sAm + k
+    st = make_map3(&tm_a, d.A, d.K, d.M, d.batch, d.sAm, d.sAz, 128);
+  if (st != MLA_OK) return st;
+  st = make_map3(&tm_b, d.B, d.K, d.N, d.batch, d.sBn, d.sBz, BN);
+  if (st != MLA_OK) return st;
+  GemmTcArgs g;
+  g.M = d.M;
+  g.N = d.N;
+  g.K = d.K;
+  g.BN = BN;
+  const int kchunks = (d.K + 63) / 64;
+  const int ntile = (d.N + BN - 1) / BN, mtile = (d.M + 127) / 128;
+  int splits = 1;
+  if (d.c_fp32 && d.allow_split) {
+    // spread long reductions over more CTAs when the tile grid is small
+    const int ctas = ntile * mtile * d.batch;
+    while (splits < 8 && ctas * splits * 2 <= 296 && kchunks / (splits * 2) >= 4) splits *= 2;
+  }
+  g.splits = splits;
+  g.k_chunks = (kchunks + splits - 1) / splits;
+  g.batch = d.batch;
+  g.a_mn = d.a_mn;
+  g.C = d.C;
+  g.sCz = d.sCz;
+  g.sCm = d.sCm;
+  g.sCn = d.sCn;
+  g.c_fp32 = d.c_fp32;
+  g.status = d.status;
+  if (splits > 1) {
+    if (!d.c_contiguous)
+      return fail(MLA_ERR_UNSUPPORTED, "split-K needs a contiguous fp32 output");
+    MLA_CUDA_TRY(cudaMemsetAsync(d.C, 0, d.c_bytes, stream));
+  }
+  MLA_CUDA_TRY(cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)kSmemBytes));
+  dim3 grid(ntile, mtile, d.batch * splits);
+  gemm_tc_kernel<<<grid, 128, kSmemBytes, stream>>>(tm_a, tm_b, g);
+  MLA_LAUNCH_CHECK("gemm_tc_kernel");
+  return MLA_OK;
+}
+
+}  // namespace mla

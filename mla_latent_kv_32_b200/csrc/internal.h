@@ -21,6 +21,27 @@ struct GemmArgs {
 };
 mla_status_t launch_gemm_simt(const GemmArgs &g, cudaStream_t stream);
 
+// Tensor-core GEMM: C[z][m][n] = sum_k A[z][m][k] * B[z][n][k].
+// A element (z,m,k): K-major at A + z*sAz + m*sAm + k, or (a_mn) MN-major at
+// A + z*sAz + k*sAk + m. B element (z,n,k) at B + z*sBz + n*sBn + k.
+// All strides in elements, multiples of 8 (16 bytes); K % 16 == 0.
+struct GemmTcDesc {
+  const uint16_t *A;
+  long long sAz, sAm, sAk;
+  int a_mn;
+  const uint16_t *B;
+  long long sBz, sBn;
+  void *C;
+  long long sCz, sCm, sCn;
+  int c_fp32;
+  int M, N, K, batch;
+  int allow_split;       // fp32 output may be split over K (atomic adds, zeroed first)
+  int c_contiguous;      // C occupies c_bytes contiguous bytes (needed for the split)
+  size_t c_bytes;
+  uint32_t *status;
+};
+mla_status_t launch_gemm_tc(const GemmTcDesc &d, cudaStream_t stream);
+
 // q_full[t][h][512:576] = RoPE(q_pe[t][h][:], pos[t]) (or copy when pos == NULL).
 mla_status_t launch_q_rope_pack(const uint16_t *q_pe, int ld_qp, const int32_t *pos,
                                 const float *rope_table, int max_pos, int T, int n_h,

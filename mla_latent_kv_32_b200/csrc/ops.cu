@@ -3,37 +3,42 @@
 
 namespace mla {
 
-// q_full[t][h][c] = sum_d q_nope[t][h][d] * w_uk[h][d][c]   (batched over heads)
+// q_full[t][h][c] = sum_d q_nope[t][h][d] * w_uk[h][d][c]   (batched over heads;
+// m = latent column c, n = token t, k = d; W^UK read as its transpose)
 mla_status_t launch_absorb_q(const uint16_t *q_nope, int ld_qn, const uint16_t *w_uk, int T,
                              int n_h, uint16_t *q_full, cudaStream_t stream) {
-  GemmArgs g;
-  g.A = q_nope; g.sAz = MLA_D_NOPE; g.sAm = ld_qn; g.sAk = 1;
-  g.B = w_uk; g.sBz = (long long)MLA_D_NOPE * MLA_D_C; g.sBn = 1; g.sBk = MLA_D_C;
-  g.C = q_full; g.sCz = MLA_ROW; g.sCm = (long long)n_h * MLA_ROW; g.sCn = 1;
-  g.c_fp32 = 0; g.M = T; g.N = MLA_D_C; g.K = MLA_D_NOPE; g.batch = n_h;
-  return launch_gemm_simt(g, stream);
+  GemmTcDesc d = {};
+  d.A = w_uk; d.sAz = (long long)MLA_D_NOPE * MLA_D_C; d.sAk = MLA_D_C; d.a_mn = 1;
+  d.B = q_nope; d.sBz = MLA_D_NOPE; d.sBn = ld_qn;
+  d.C = q_full; d.sCz = MLA_ROW; d.sCm = 1; d.sCn = (long long)n_h * MLA_ROW;
+  d.c_fp32 = 0; d.M = MLA_D_C; d.N = T; d.K = MLA_D_NOPE; d.batch = n_h;
+  return launch_gemm_tc(d, stream);
 }
 
-// u[t][h*128 + d] = sum_c o[t][h][c] * w_uv[h][d][c]   (batched over heads)
+// u[t][h*128 + d] = sum_c o[t][h][c] * w_uv[h][d][c]   (batched over heads;
+// m = d, n = token t, k = c)
 mla_status_t launch_out_absorb(const uint16_t *o_latent, const uint16_t *w_uv, int T, int n_h,
                                uint16_t *u, int ld_u, cudaStream_t stream) {
-  GemmArgs g;
-  g.A = o_latent; g.sAz = MLA_D_C; g.sAm = (long long)n_h * MLA_D_C; g.sAk = 1;
-  g.B = w_uv; g.sBz = (long long)MLA_D_V * MLA_D_C; g.sBn = MLA_D_C; g.sBk = 1;
-  g.C = u; g.sCz = MLA_D_V; g.sCm = ld_u; g.sCn = 1;
-  g.c_fp32 = 0; g.M = T; g.N = MLA_D_V; g.K = MLA_D_C; g.batch = n_h;
-  return launch_gemm_simt(g, stream);
+  GemmTcDesc d = {};
+  d.A = w_uv; d.sAz = (long long)MLA_D_V * MLA_D_C; d.sAm = MLA_D_C; d.a_mn = 0;
+  d.B = o_latent; d.sBz = MLA_D_C; d.sBn = (long long)n_h * MLA_D_C;
+  d.C = u; d.sCz = MLA_D_V; d.sCm = 1; d.sCn = ld_u;
+  d.c_fp32 = 0; d.M = MLA_D_V; d.N = T; d.K = MLA_D_C; d.batch = n_h;
+  return launch_gemm_tc(d, stream);
 }
 
-// C[m][n] = sum_k X[m][k] * W[n][k]
+// C[t][f] = sum_k X[t][k] * W[f][k]   (m = output feature f, n = token t)
 mla_status_t launch_projection(const uint16_t *X, int ld_x, const uint16_t *W, int ld_w, void *C,
                                int ld_c, int c_fp32, int M, int N, int K, cudaStream_t stream) {
-  GemmArgs g;
-  g.A = X; g.sAz = 0; g.sAm = ld_x; g.sAk = 1;
-  g.B = W; g.sBz = 0; g.sBn = ld_w; g.sBk = 1;
-  g.C = C; g.sCz = 0; g.sCm = ld_c; g.sCn = 1;
-  g.c_fp32 = c_fp32; g.M = M; g.N = N; g.K = K; g.batch = 1;
-  return launch_gemm_simt(g, stream);
+  GemmTcDesc d = {};
+  d.A = W; d.sAz = 0; d.sAm = ld_w; d.a_mn = 0;
+  d.B = X; d.sBz = 0; d.sBn = ld_x;
+  d.C = C; d.sCz = 0; d.sCm = 1; d.sCn = ld_c;
+  d.c_fp32 = c_fp32; d.M = N; d.N = M; d.K = K; d.batch = 1;
+  d.allow_split = c_fp32;
+  d.c_contiguous = 1;
+  d.c_bytes = (size_t)M * ld_c * (c_fp32 ? 4 : 2);
+  return launch_gemm_tc(d, stream);
 }
 
 mla_status_t launch_decode(const DecodeArgs &a, cudaStream_t stream) {

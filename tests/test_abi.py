@@ -54,7 +54,7 @@ def test_invalid_arguments_rejected_before_launch(lib):
         mla.mla_absorb_q(16, 2048, 16, 1024, 16, None, None, 0, 1, 24, 16, stream=0)
     assert e.value.status == mla.MLA_ERR_UNSUPPORTED
     with pytest.raises(mla.MlaError) as e:
-        mla.mla_gemm_bf16(16, 8, 16, 8, 8, 8, 0, 4, 4, 8, stream=0)   # C misaligned
+        mla.mla_gemm_bf16(16, 16, 16, 16, 8, 16, 0, 4, 4, 16, stream=0)   # C misaligned
     assert e.value.status == mla.MLA_ERR_INVALID_ARGUMENT
     # zero-sized calls are no-ops that succeed without a device
     mla.mla_cache_append(None, 1, None, 1, 1, None, None, None, 512, None, 64, None, 1, 0, stream=0)
