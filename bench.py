@@ -43,8 +43,11 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # DRAM traffic per launch of mla_decode_attention measured by ncu
 # (dram__bytes_read.sum + dram__bytes_write.sum), keyed by the SHA-256 of the
-# decode sources it was measured on; reported only while the sources match.
-TRAFFIC = {}
+# decode sources it was measured on and the workload; reported only while the
+# sources match (the combine kernel's few MB are not included).
+TRAFFIC = {
+    ("8f2878d6b69bf07b", "v3"): 333660672,   # decode_tc_kernel
+}
 
 
 def parse():
@@ -212,6 +215,22 @@ def run_reference(args, rank, world):
     return 0
 
 
+def max_over_ranks(values, dist, device, world):
+    """Element-wise maximum of per-rank timings (the slowest rank sets the job
+    time). ``dist`` is torch.distributed; with one rank it is not touched."""
+    import torch
+    if world <= 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def whole_job_rate(world, units_per_rank, t_ms):
+    """Units processed by all ranks per second, given the max-over-ranks time."""
+    return world * units_per_rank / (t_ms / 1e3)
+
+
 def workload_config(w, inp, sess):
     cfg = {"workload": f"{w.name}: absorbed MLA decode, batch {w.B}, {w.q_len} query token(s) "
                        f"per sequence, context {'U[1,%d]' % w.L if w.lens == 'ragged' else w.L}, "
@@ -292,13 +311,10 @@ def main():
     attn_ms = [e[1].elapsed_time(e[2]) for e in ev]
     t_step = sum(step_ms) / K
     t_attn = sum(attn_ms) / K
-    if world > 1:
-        t = torch.tensor([t_step, t_attn], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        t_step, t_attn = float(t[0]), float(t[1])
+    t_step, t_attn = max_over_ranks([t_step, t_attn], dist, dev, world)
 
     tokens = w.B * w.q_len
-    value = world * tokens / (t_step / 1e3)
+    value = whole_job_rate(world, tokens, t_step)
     cache_bytes = int(inp.lens.sum()) * ROW_BYTES
     # FLOPs: 2176 per (visible cached token, head, query)
     vis = sum(int(L) - w.q_len + j + 1 for L in inp.lens for j in range(w.q_len))
@@ -322,11 +338,8 @@ def main():
             ee[k][1].record(stream)
         barrier()
         t_e2e = sum(a.elapsed_time(b) for a, b in ee) / K
-        if world > 1:
-            t = torch.tensor([t_e2e], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            t_e2e = float(t[0])
-        e2e = {"value": world * tokens / (t_e2e / 1e3), "unit": UNIT,
+        (t_e2e,) = max_over_ranks([t_e2e], dist, dev, world)
+        e2e = {"value": whole_job_rate(world, tokens, t_e2e), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": t_e2e}
 
@@ -336,7 +349,7 @@ def main():
     t_mem = cache_bytes / (peaks["hbm_gbs"] * 1e9)
     t_tc = flops / (peaks["bf16_tflops"] * 1e12)
     src_hash = decode_sources_hash()
-    traffic = TRAFFIC.get(src_hash)
+    traffic = TRAFFIC.get((src_hash, args.workload))
     roof = {
         "kernel": "mla_decode_attention (decode + combine kernels)",
         "bound": "hbm" if t_mem >= t_tc else "tensor",
