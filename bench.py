@@ -45,9 +45,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # (dram__bytes_read.sum + dram__bytes_write.sum), keyed by the SHA-256 of the
 # decode sources it was measured on and the workload; reported only while the
 # sources match (the combine kernel's few MB are not included).
-TRAFFIC = {
-    ("8f2878d6b69bf07b", "v3"): 333660672,   # decode_tc_kernel
-}
+TRAFFIC = {}
 
 
 def parse():
@@ -58,7 +56,7 @@ def parse():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--workload", default="v3")
     ap.add_argument("--num-ctas", type=int, default=0)
-    ap.add_argument("--max-split", type=int, default=0)
+    ap.add_argument("--max-split", type=int, default=-1)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     return ap.parse_args()

@@ -163,7 +163,11 @@ size_t mla_plan_bytes(int batch, int q_len, int num_ctas);
  *             q_len new ones (1 <= q_len <= seq_lens[b]).
  *   num_ctas: work lists to balance over; 0 = derive from the current
  *             device's SM count.
- *   max_split: upper bound on the items one (sequence, query) is cut into; 0 = no bound.
+ *   max_split: 1 = every (sequence, query) is one item (no combine pass);
+ *             0 = cut the pages of all sequences into num_ctas equal ranges
+ *             (long sequences become several items merged by the combine);
+ *             negative = build both and keep the one with the smaller
+ *             estimated time.
  *   plan:     host buffer of plan_bytes (>= mla_plan_bytes(batch, q_len, num_ctas)).
  *   info:     out, may be NULL.
  * Errors: INVALID_ARGUMENT (bad lengths), WORKSPACE_TOO_SMALL (plan buffer).

@@ -70,12 +70,17 @@ def build(verbose: bool = False, force: bool = False, extra_flags=None) -> str:
 
     with ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
         list(ex.map(run, jobs))
-    relink = jobs or not os.path.exists(LIB) or any(
+    # relink when an object changed or the set of sources did (a removed .cu)
+    manifest = os.path.join(BUILD, "objects.txt")
+    listed = open(manifest).read() if os.path.exists(manifest) else ""
+    relink = jobs or not os.path.exists(LIB) or listed != "\n".join(objs) or any(
         os.path.getmtime(o) > os.path.getmtime(LIB) for o in objs)
     if relink:
         tmp = LIB + ".tmp"
         run([nvcc()] + ARCH + ["-shared", "-o", tmp] + objs + ["-lpthread"])
         os.replace(tmp, LIB)
+        with open(manifest, "w") as f:
+            f.write("\n".join(objs))
     return LIB
 
 

@@ -171,7 +171,6 @@ mla_status_t mla_decode_plan(const int32_t *seq_lens, int batch, int q_len, int 
     return fail(MLA_ERR_UNSUPPORTED, "n_h = %d (supported: 16..128, multiple of 16)", n_h);
   MLA_CHECK_ARG(batch == 0 || seq_lens != nullptr, "seq_lens is NULL");
   MLA_CHECK_ARG(plan != nullptr, "plan is NULL");
-  MLA_CHECK_ARG(max_split >= 0, "max_split < 0");
   mla_status_t st = resolve_ctas(&num_ctas);
   if (st != MLA_OK) return st;
   const size_t need = plan_bytes_for(batch, q_len, num_ctas);
@@ -195,19 +194,19 @@ mla_status_t mla_decode_plan(const int32_t *seq_lens, int batch, int q_len, int 
       total += pages;
       max_unit = std::max(max_unit, pages);
     }
-  // Work lists. With max_split == 1 every (sequence, query) is one item and
-  // items go to lists by longest-processing-time order. Otherwise the units'
-  // pages are laid end to end and cut into num_ctas near-equal ranges, so
-  // every list carries the same page count; a unit crossing a cut becomes
-  // several items whose partial results the combine pass merges. Adjacent
-  // units (the two queries of an MTP step) start on neighbouring lists at the
-  // same time, so their shared pages are read once from HBM and once from L2.
-  std::vector<std::vector<WorkItem>> per;
-  std::vector<CombineItem> comb;
-  int slots = 0;
+  // Work lists. The "whole" plan makes every (sequence, query) one item and
+  // deals the items to lists in longest-processing-time order. The "cut" plan
+  // lays the units' pages end to end and cuts them into num_ctas near-equal
+  // ranges, so every list carries the same page count; a unit crossing a cut
+  // becomes several items whose partial results the combine pass merges.
+  // Adjacent units (the two queries of an MTP step) start on neighbouring
+  // lists at the same time, so their shared pages are read once from HBM and
+  // once from L2. max_split == 1 selects the whole plan, max_split >= 0 the
+  // cut plan, max_split < 0 the one with the smaller estimated time.
   int max_pages_used = 0;
   for (const Unit &u : units) max_pages_used = std::max(max_pages_used, u.pages);
-  if (max_split == 1) {
+  typedef std::vector<std::vector<WorkItem>> Lists;
+  auto plan_whole = [&](Lists &per) {
     std::vector<int> order(units.size());
     for (size_t i = 0; i < order.size(); ++i) order[i] = (int)i;
     std::stable_sort(order.begin(), order.end(),
@@ -225,7 +224,8 @@ mla_status_t mla_decode_plan(const int32_t *seq_lens, int batch, int q_len, int 
       ld.first += u.pages;
       heap.push(ld);
     }
-  } else {
+  };
+  auto plan_cut = [&](Lists &per, std::vector<CombineItem> &comb, int &slots) {
     const int lists = (int)std::max<long long>(1, std::min<long long>(num_ctas, total));
     const long long target = (total + lists - 1) / lists;
     per.assign(lists, {});
@@ -252,6 +252,35 @@ mla_status_t mla_decode_plan(const int32_t *seq_lens, int batch, int q_len, int 
           per[where[p].first][where[p].second].slot = slots + (int)p;
         slots += (int)where.size();
       }
+    }
+  };
+  // Estimated time of a plan in units of one score/output tile (4 pages): the
+  // busiest list's tiles plus a fixed cost per item (query load, pipeline
+  // refill, epilogue) and, when parts must be merged, the combine pass.
+  auto estimate = [&](const Lists &per, bool merged) {
+    long long worst = 0;
+    for (const auto &v : per) {
+      long long t = 0;
+      for (const WorkItem &it : v) t += (it.page_end - it.page_begin + 3) / 4 + 2;
+      worst = std::max(worst, t);
+    }
+    return worst + (merged ? 2 : 0);
+  };
+  Lists per;
+  std::vector<CombineItem> comb;
+  int slots = 0;
+  if (max_split == 1) {
+    plan_whole(per);
+  } else if (max_split >= 0) {
+    plan_cut(per, comb, slots);
+  } else {
+    Lists whole;
+    plan_whole(whole);
+    plan_cut(per, comb, slots);
+    if (estimate(whole, false) <= estimate(per, !comb.empty())) {
+      per.swap(whole);
+      comb.clear();
+      slots = 0;
     }
   }
   size_t n_items = 0;

@@ -71,7 +71,7 @@ struct DecodeArgs {
   uint32_t *status;
 };
 mla_status_t launch_decode_simt(const DecodeArgs &a, cudaStream_t stream);
-mla_status_t launch_decode_tc(const DecodeArgs &a, cudaStream_t stream);
+mla_status_t launch_decode_pair(const DecodeArgs &a, cudaStream_t stream);
 mla_status_t launch_combine(const DecodeArgs &a, cudaStream_t stream);
 
 // The kernels behind each entry point (ops.cu).

@@ -42,7 +42,7 @@ mla_status_t launch_projection(const uint16_t *X, int ld_x, const uint16_t *W, i
 }
 
 mla_status_t launch_decode(const DecodeArgs &a, cudaStream_t stream) {
-  return launch_decode_tc(a, stream);
+  return launch_decode_pair(a, stream);
 }
 
 }  // namespace mla

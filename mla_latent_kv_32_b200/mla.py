@@ -145,7 +145,7 @@ def mla_plan_bytes(batch: int, q_len: int, num_ctas: int = 0) -> int:
 
 
 def mla_decode_plan(seq_lens: np.ndarray, batch: int, q_len: int, n_h: int, num_ctas: int = 0,
-                    max_split: int = 0):
+                    max_split: int = -1):
     """Returns (plan bytes as a uint8 numpy array, mla_plan_info_t)."""
     lens = np.ascontiguousarray(seq_lens, dtype=np.int32)
     nbytes = mla_plan_bytes(batch, q_len, num_ctas)

@@ -43,7 +43,7 @@ class DecodeSession:
         mla_out_absorb   (u = W^UV o)
     """
 
-    def __init__(self, inp, device="cuda", num_ctas: int = 0, max_split: int = 0,
+    def __init__(self, inp, device="cuda", num_ctas: int = 0, max_split: int = -1,
                  scale: float = DEFAULT_SCALE, rope_table: Optional[np.ndarray] = None):
         w = inp.w
         self.w = w
@@ -140,7 +140,7 @@ class LayerSession:
     The rows of h that are queries must be the last B*q_len rows.
     """
 
-    def __init__(self, inp, device="cuda", num_ctas: int = 0, max_split: int = 0,
+    def __init__(self, inp, device="cuda", num_ctas: int = 0, max_split: int = -1,
                  scale: float = DEFAULT_SCALE):
         w = inp.w
         self.w = w

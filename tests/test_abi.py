@@ -139,6 +139,15 @@ def test_planner_no_split_mode():
     assert max(loads) == 64
 
 
+def test_planner_auto_picks_by_estimate():
+    # equal lengths that fill most lists: one item per sequence, no combine
+    p, loads, total = check_plan([4096] * 64, 1, 74, max_split=-1)
+    assert p["num_partials"] == 0 and p["num_items"] == 64
+    # a few very long sequences: cut, merged by the combine pass
+    p, loads, total = check_plan([131072] * 4, 2, 74, max_split=-1)
+    assert p["num_partials"] > 0 and max(loads) <= -(-total // 74)
+
+
 def test_planner_rejects_bad_input():
     with pytest.raises(mla.MlaError):
         mla.mla_decode_plan(np.array([1, 0], np.int32), 2, 1, 128, 8)    # L < q_len
