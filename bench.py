@@ -45,7 +45,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # (dram__bytes_read.sum + dram__bytes_write.sum), keyed by the SHA-256 of the
 # decode sources it was measured on and the workload; reported only while the
 # sources match (the combine kernel's few MB are not included).
-TRAFFIC = {}
+TRAFFIC = {
+    ("e3c8d0931702c06a", "v3"): 317871616,   # decode_pair_kernel
+}
 
 
 def parse():

@@ -226,25 +226,38 @@ mla_status_t mla_decode_plan(const int32_t *seq_lens, int batch, int q_len, int 
     }
   };
   auto plan_cut = [&](Lists &per, std::vector<CombineItem> &comb, int &slots) {
+    // Cuts fall on 4-page boundaries of each unit (the kernels' tile), so a
+    // split adds no partial tile. List c ends near the cumulative boundary
+    // total * (c + 1) / lists: a tile joins the list unless it would overshoot
+    // the boundary by more than half its size, so lists differ by about one
+    // tile and the rounding does not drift onto the last list.
     const int lists = (int)std::max<long long>(1, std::min<long long>(num_ctas, total));
-    const long long target = (total + lists - 1) / lists;
+    auto boundary = [&](int c) { return (total * (c + 1) + lists / 2) / lists; };
     per.assign(lists, {});
     int c = 0;
-    long long fill = 0;
+    long long fill = 0, cum = 0;
     for (const Unit &u : units) {
-      int begin = 0;
       std::vector<std::pair<int, int>> where;  // (list, index in list)
+      int begin = 0;
       while (begin < u.pages) {
-        if (fill >= target && c < lists - 1) {
+        int end = begin;
+        while (end < u.pages) {
+          const int tile = std::min(4, u.pages - end);
+          const bool over = c < lists - 1 && 2 * (cum + tile) > 2 * boundary(c) + tile;
+          if (over && fill > 0) break;
+          end += tile;
+          cum += tile;
+          fill += tile;
+        }
+        if (end > begin) {
+          where.push_back({c, (int)per[c].size()});
+          per[c].push_back(WorkItem{u.b, u.j, begin, end, -1, u.L, u.qpos, 0});
+          begin = end;
+        }
+        if (begin < u.pages) {  // list c is full
           ++c;
           fill = 0;
         }
-        const int take = (int)std::min<long long>(u.pages - begin,
-                                                  c < lists - 1 ? target - fill : u.pages - begin);
-        where.push_back({c, (int)per[c].size()});
-        per[c].push_back(WorkItem{u.b, u.j, begin, begin + take, -1, u.L, u.qpos, 0});
-        begin += take;
-        fill += take;
       }
       if (where.size() > 1) {
         comb.push_back(CombineItem{u.b, u.j, slots, (int)where.size()});

@@ -121,16 +121,21 @@ def check_plan(lens, q_len, num_ctas, max_split=0, n_h=128):
     ([4096] * 64, 1, 74), ([1, 63, 64, 65, 127, 200], 1, 3), ([2, 131072, 5000, 64], 2, 74),
     ([1], 1, 74), ([300] * 7, 2, 1)])
 def test_planner_contiguous_cuts(lens, q_len, ctas):
-    p, loads, total = check_plan(lens, q_len, ctas)
-    assert max(loads) <= -(-total // min(ctas, total))
+    p, loads, total = check_plan(lens, q_len, ctas, max_split=0)
+    # cuts fall on 4-page tiles: a list exceeds its equal share by under a tile
+    assert max(loads) <= -(-total // min(ctas, total)) + 3
+    # every cut inside a unit is tile-aligned
+    for it in p["items"]:
+        assert it["page_begin"] % 4 == 0
 
 
 def test_planner_ragged_workload_balanced():
     import synth
     w = synth.WORKLOADS["ragged"]
     lens = synth.seq_lens(w)
-    p, loads, total = check_plan(lens, 1, 74)
-    assert max(loads) - min(loads) <= 1 or max(loads) <= -(-total // 74)
+    p, loads, total = check_plan(lens, 1, 74, max_split=0)
+    # the cut plan balances pages to within a tile of the equal share
+    assert max(loads) <= -(-total // 74) + 3 and min(loads) >= total // 74 - 4
 
 
 def test_planner_no_split_mode():
@@ -145,7 +150,7 @@ def test_planner_auto_picks_by_estimate():
     assert p["num_partials"] == 0 and p["num_items"] == 64
     # a few very long sequences: cut, merged by the combine pass
     p, loads, total = check_plan([131072] * 4, 2, 74, max_split=-1)
-    assert p["num_partials"] > 0 and max(loads) <= -(-total // 74)
+    assert p["num_partials"] > 0 and max(loads) <= -(-total // 74) + 3
 
 
 def test_planner_rejects_bad_input():
