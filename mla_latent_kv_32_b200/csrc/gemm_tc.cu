@@ -13,8 +13,10 @@
 // A (the weight) is K-major or MN-major in global memory, B (the activations)
 // is K-major; both arrive through 3-D TMA tensor maps (z = head or split) in
 // 64-element k-chunks with the 128-byte swizzle. One CTA computes one
-// 128 x BN tile: warp 0 lane 0 issues TMA into a 4-stage ring, warp 1 lane 0
-// issues the MMAs into a TMEM accumulator, all four warps then read it back
+// 128 x BN tile: warp 0 lane 0 issues TMA into a ring of up to 4 stages, warp
+// 1 lane 0 issues the MMAs into a TMEM accumulator of BN columns (shared memory
+// and TMEM are sized to the tile, so several CTAs share an SM when the tiles
+// are small), all four warps then read it back
 // (thread = row m) and write C through arbitrary strides, as bf16 or fp32
 // (fp32 outputs may be split over K and reduced with atomic adds).
 #include <cuda.h>
@@ -28,17 +30,16 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kStages = 4;
+constexpr int kMaxStages = 4;
 constexpr uint32_t kAStage = 128 * 128;        // 128 rows x 64 k (bf16) = 16 KB
-constexpr uint32_t kBStageMax = 256 * 128;     // up to 256 rows x 64 k = 32 KB
-constexpr uint32_t kStageBytes = kAStage + kBStageMax;
-constexpr uint32_t kOffBar = kStages * kStageBytes;  // 196608
-constexpr uint32_t kSmemBytes = kOffBar + 128 + 1024;
 constexpr uint64_t kTimeoutNs = 1000000000ull;
 
 struct GemmTcArgs {
   int M, N, K;          // per batch
   int BN;               // tile width in n (multiple of 16, <= 256)
+  int stages;           // ring depth (1..kMaxStages)
+  uint32_t stage_bytes; // A chunk + B chunk, rounded to 1 KB
+  uint32_t tmem_cols;   // accumulator columns allocated (power of two >= BN, >= 32)
   int k_chunks;         // 64-element k-chunks per split
   int splits;           // split-K factor (fp32 output only)
   int batch;
@@ -61,7 +62,7 @@ __device__ __noinline__ bool wait_bar_g(uint32_t bar, uint32_t parity, uint32_t 
   }
 }
 
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(128, 4)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                const GemmTcArgs g) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -75,19 +76,20 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__
   const int split = blockIdx.z % g.splits;
   const int kc0 = split * g.k_chunks;
   const int kc1 = min(kc0 + g.k_chunks, (g.K + 63) / 64);
-  const uint32_t bar_full = base + kOffBar, bar_empty = bar_full + 8 * kStages;
-  const uint32_t bar_done = bar_empty + 8 * kStages, tptr = bar_done + 8;
+  const int stages = g.stages;
+  const uint32_t bar_full = base + stages * g.stage_bytes, bar_empty = bar_full + 8 * kMaxStages;
+  const uint32_t bar_done = bar_empty + 8 * kMaxStages, tptr = bar_done + 8;
   const uint32_t b_bytes = (uint32_t)g.BN * 128;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kStages; ++i) {
+    for (int i = 0; i < stages; ++i) {
       mbar_init(bar_full + 8 * i, 1);
       mbar_init(bar_empty + 8 * i, 1);
     }
     mbar_init(bar_done, 1);
     fence_mbar_init_cluster();
   }
-  if (warp == 1) tmem_alloc(tptr, 256);
+  if (warp == 1) tmem_alloc(tptr, g.tmem_cols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -96,12 +98,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tm_a);
     tma_prefetch_desc(&tm_b);
-    int armed[kStages] = {};
+    int armed[kMaxStages] = {};
     for (int kc = kc0, i = 0; kc < kc1; ++kc, ++i) {
-      const int s = i % kStages;
-      if (i >= kStages && !wait_bar_g(bar_empty + 8 * s, ((i / kStages) - 1) & 1, g.status))
+      const int s = i % stages;
+      if (i >= stages && !wait_bar_g(bar_empty + 8 * s, ((i / stages) - 1) & 1, g.status))
         break;
-      const uint32_t a_s = base + s * kStageBytes, b_s = a_s + kAStage;
+      const uint32_t a_s = base + s * g.stage_bytes, b_s = a_s + kAStage;
       mbar_arrive_expect_tx(bar_full + 8 * s, kAStage + b_bytes);
       ++armed[s];
       if (g.a_mn) {
@@ -113,15 +115,15 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__
       }
       tma_load_3d(b_s, &tm_b, kc * 64, n0, z, bar_full + 8 * s);
     }
-    for (int s = 0; s < kStages; ++s)
+    for (int s = 0; s < stages; ++s)
       if (armed[s]) wait_bar_g(bar_full + 8 * s, (armed[s] - 1) & 1, g.status);
   } else if (warp == 1 && lane == 0) {
     const uint32_t idesc = idesc_bf16(128, g.BN, g.a_mn, 0);
     for (int kc = kc0, i = 0; kc < kc1; ++kc, ++i) {
-      const int s = i % kStages;
-      if (!wait_bar_g(bar_full + 8 * s, (i / kStages) & 1, g.status)) break;
+      const int s = i % stages;
+      if (!wait_bar_g(bar_full + 8 * s, (i / stages) & 1, g.status)) break;
       tc_fence_after();
-      const uint32_t a_s = base + s * kStageBytes, b_s = a_s + kAStage;
+      const uint32_t a_s = base + s * g.stage_bytes, b_s = a_s + kAStage;
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {
         const uint64_t ad = g.a_mn ? smem_desc(a_s + kk * 2048, 8192, 1024, kSwizzle128B)
@@ -164,7 +166,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, g.tmem_cols);
   }
 }
 
@@ -230,6 +232,11 @@ mla_status_t launch_gemm_tc(const GemmTcDesc &d, cudaStream_t stream) {
   }
   g.splits = splits;
   g.k_chunks = (kchunks + splits - 1) / splits;
+  g.stages = g.k_chunks < kMaxStages ? g.k_chunks : kMaxStages;
+  g.stage_bytes = kAStage + (((uint32_t)BN * 128 + 1023u) & ~1023u);
+  g.tmem_cols = 32;
+  while (g.tmem_cols < (uint32_t)BN) g.tmem_cols *= 2;
+  const uint32_t smem_bytes = g.stages * g.stage_bytes + 8 * (2 * kMaxStages + 2) + 1024;
   g.batch = d.batch;
   g.a_mn = d.a_mn;
   g.C = d.C;
@@ -244,9 +251,9 @@ mla_status_t launch_gemm_tc(const GemmTcDesc &d, cudaStream_t stream) {
     MLA_CUDA_TRY(cudaMemsetAsync(d.C, 0, d.c_bytes, stream));
   }
   MLA_CUDA_TRY(cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    (int)kSmemBytes));
+                                    (int)smem_bytes));
   dim3 grid(ntile, mtile, d.batch * splits);
-  gemm_tc_kernel<<<grid, 128, kSmemBytes, stream>>>(tm_a, tm_b, g);
+  gemm_tc_kernel<<<grid, 128, smem_bytes, stream>>>(tm_a, tm_b, g);
   MLA_LAUNCH_CHECK("gemm_tc_kernel");
   return MLA_OK;
 }
