@@ -320,28 +320,40 @@ def main():
     vis = sum(int(L) - w.q_len + j + 1 for L in inp.lens for j in range(w.q_len))
     flops = float(vis) * w.n_h * FLOP_PER_TOKEN_HEAD
 
-    # e2e: per-step inputs from pinned host memory, result read back
+    # e2e: per-step inputs from pinned host memory, result read back to pinned
+    # host memory, through the library's calls. Two independent sessions
+    # (each with its own 302 MB cache, weights and I/O buffers) alternate
+    # steps, so one batch's uploads and downloads overlap the other's compute;
+    # every step touches more than L2 holds, so no flush runs in this loop.
     e2e = None
     if not args.no_e2e:
-        ins, host_in, host_out = sess.pinned_step_buffers()
-        h2d, d2h = DecodeSession.step_io_bytes(ins, host_out)
-        for _ in range(3):
-            sess.step_e2e(ins, host_in, host_out)
+        from mla_latent_kv_32_b200.runtime import run_e2e_pipelined
+        sess2 = DecodeSession(inp, dev, num_ctas=args.num_ctas, max_split=args.max_split)
+        pair = [sess, sess2]
+        for s_ in pair:
+            s_.capture()   # one graph launch per step: the loop is not bound by host launches
+        ins, host_in, host_out0 = sess.pinned_step_buffers()
+        host_outs = [host_out0, torch.empty_like(host_out0).pin_memory()]
+        h2d, d2h = DecodeSession.step_io_bytes(ins, host_out0)
+        comp = torch.cuda.current_stream()
+        up_s, down_s = torch.cuda.Stream(), torch.cuda.Stream()
+        run_e2e_pipelined(pair, host_in, host_outs, 4, comp, up_s, down_s)
         torch.cuda.synchronize()
-        ee = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(K)]
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         barrier()
-        for k in range(K):
-            flush.zero_()
-            ee[k][0].record(stream)
-            sess.step_e2e(ins, host_in, host_out)
-            ee[k][1].record(stream)
+        e0.record(comp)
+        run_e2e_pipelined(pair, host_in, host_outs, K, comp, up_s, down_s)
+        e1.record(comp)
         barrier()
-        t_e2e = sum(a.elapsed_time(b) for a, b in ee) / K
+        t_e2e = e0.elapsed_time(e1) / K
         (t_e2e,) = max_over_ranks([t_e2e], dist, dev, world)
         e2e = {"value": whole_job_rate(world, tokens, t_e2e), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-               "ms_per_step": t_e2e}
+               "ms_per_step": t_e2e,
+               "method": "two sessions alternate steps (each step one CUDA graph of the four "
+                         "library calls); uploads and downloads overlap the other batch's "
+                         "compute; no L2 flush (each step touches > L2)"}
+        del sess2
 
     peaks, peak_src = load_peaks()
     gbs = cache_bytes / (t_attn / 1e3) / 1e9

@@ -109,7 +109,29 @@ class DecodeSession:
     def read_status(self) -> int:
         return mla.mla_read_status(self.status, clear=True)
 
+    def capture(self):
+        """Record one step (the four library calls, fixed buffers and plan) in
+        a CUDA graph; ``replay(stream)`` then runs it as a single launch."""
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            self.step(side)
+        torch.cuda.current_stream().wait_stream(side)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=side):
+            self.step(side)
+        self.graph = g
+        return g
+
+    def replay(self, stream):
+        with torch.cuda.stream(stream):
+            self.graph.replay()
+
     # e2e: per-step inputs from pinned host memory, result back to host ----
+    def io_inputs(self):
+        """Device tensors a step reads that come from the host each step."""
+        return [self.q_nope, self.q_pe, self.c_new, self.k_new]
+
     def pinned_step_buffers(self):
         """Pinned host copies of the per-step inputs and of the result."""
         ins = [self.q_nope, self.q_pe, self.c_new, self.k_new]
@@ -127,6 +149,56 @@ class DecodeSession:
     def step_io_bytes(ins, host_out) -> tuple:
         return (sum(t.numel() * t.element_size() for t in ins),
                 host_out.numel() * host_out.element_size())
+
+
+def run_e2e_pipelined(sessions, host_in, host_outs, steps, comp, h2d, d2h):
+    """End-to-end decode steps with host I/O overlapped across independent batches.
+
+    Step k runs on sessions[k % len(sessions)] (each owns its cache, weights,
+    plan and device I/O buffers): the upload of step k+1's inputs (pinned
+    ``host_in``, one list of tensors matching each session's ``io_inputs()``)
+    runs on ``h2d`` while step k computes on ``comp``, and the download of
+    step k's result ``u`` into ``host_outs[k % len(sessions)]`` runs on ``d2h``
+    while step k+1 computes. Every step still moves its inputs host->device and
+    its result device->host; ``comp`` waits for the last download at the end.
+    """
+    n = len(sessions)
+    up = [torch.cuda.Event() for _ in range(n)]
+    done = [torch.cuda.Event() for _ in range(n)]
+    down = [torch.cuda.Event() for _ in range(n)]
+    issued_down = [False] * n
+
+    def upload(k):
+        s = k % n
+        with torch.cuda.stream(h2d):
+            if k >= n:
+                h2d.wait_event(done[s])       # the session's previous step read its inputs
+            for d, h in zip(sessions[s].io_inputs(), host_in):
+                d.copy_(h, non_blocking=True)
+            up[s].record(h2d)
+
+    if steps > 0:
+        upload(0)
+    for k in range(steps):
+        s = k % n
+        if k + 1 < steps:
+            upload(k + 1)
+        comp.wait_event(up[s])
+        if issued_down[s]:
+            comp.wait_event(down[s])          # the previous download of this u finished
+        if getattr(sessions[s], "graph", None) is not None:
+            sessions[s].replay(comp)
+        else:
+            sessions[s].step(comp)
+        done[s].record(comp)
+        with torch.cuda.stream(d2h):
+            d2h.wait_event(done[s])
+            host_outs[s].copy_(sessions[s].u, non_blocking=True)
+            down[s].record(d2h)
+        issued_down[s] = True
+    for s in range(n):
+        if issued_down[s]:
+            comp.wait_event(down[s])
 
 
 class LayerSession:

@@ -122,6 +122,36 @@ def test_split_invariance(dev, num_ctas, max_split):
     check_session(sess, inp, list(range(w.B)), table, nonabs=1)
 
 
+def test_e2e_pipelined_matches_oracle(dev):
+    # the benchmark's end-to-end loop: two sessions alternate steps, uploads
+    # and downloads overlap the other batch's compute; every step's result
+    # read back to the host must be the oracle's
+    from mla_latent_kv_32_b200.runtime import run_e2e_pipelined
+    lens = [700, 64, 1, 129]
+    w = synth.Workload("e2e", B=len(lens), q_len=1, L=max(lens), n_h=128, seed=5)
+    inp = synth.make_decode_inputs(w, lens=lens)
+    table = O.rope_table(max(lens))
+    pair = [DecodeSession(inp, dev, rope_table=table) for _ in range(2)]
+    ins, host_in, host_out0 = pair[0].pinned_step_buffers()   # the true inputs
+    for s in pair:   # clobber the device inputs: the loop must upload them
+        for t in s.io_inputs():
+            t.zero_()
+    pair[1].capture()   # one session eager, one replaying a captured graph
+    for t in pair[1].io_inputs():
+        t.zero_()
+    host_outs = [torch.full_like(host_out0, 7.0).pin_memory() for _ in range(2)]
+    comp = torch.cuda.current_stream()
+    run_e2e_pipelined(pair, host_in, host_outs, 5, comp, torch.cuda.Stream(), torch.cuda.Stream())
+    torch.cuda.synchronize()
+    for s in pair:
+        assert s.read_status() == 0
+    for h in host_outs:
+        u = h.float().numpy().reshape(w.B, 1, 128, 128)
+        got = [u[b] for b in range(w.B)]
+        ref = [oracle_seq(inp, b, table)["u"] for b in range(w.B)]
+        assert_parity(np.stack(got), np.stack(ref), "u (e2e)")
+
+
 def test_bad_page_sets_status(dev):
     lens = [300, 200]
     w = synth.Workload("bad", B=2, q_len=1, L=300, n_h=128, seed=3)
