@@ -2,7 +2,8 @@
  * mla_debug.h -- diagnostic entry points of the MLA decode library.
  *
  * Not part of the decode path. They exist so that tests can compare two
- * independent GPU implementations of the same operation.
+ * independent GPU implementations of the same operation, and exercise the
+ * device-side failure detection without faulting the GPU.
  */
 #ifndef MLA_DEBUG_H_
 #define MLA_DEBUG_H_
@@ -28,6 +29,21 @@ mla_status_t mla_decode_attention_cudacore(const mla_bf16_t *q_full, const mla_b
                                            const void *plan_dev, void *workspace,
                                            size_t workspace_bytes, mla_bf16_t *o_latent,
                                            float *lse, uint32_t *status, mla_stream_t stream);
+
+/*
+ * mla_debug_decode_wait -- host. Failure-detection switch of the tensor-core
+ * decode kernel for the calls that follow (process-wide; not thread-safe).
+ *   wait_cap_seconds: bound of every wait of the decode kernel on a barrier
+ *                     (default 1.0; must be > 0 and <= 10).
+ *   suppress_arrive:  1 = the producer of each CTA pair skips its first
+ *                     arrival on the first stage barrier, so the MMA issuer's
+ *                     wait on it can only end by running out; 0 = normal.
+ * When a wait runs out the kernel sets MLA_DEV_TIMEOUT in the status word,
+ * stops issuing work, lets what it issued complete and exits; the context
+ * stays usable. The pages describe no failure handling; this is the build's
+ * own test hook. Returns INVALID_ARGUMENT for a cap outside (0, 10].
+ */
+mla_status_t mla_debug_decode_wait(double wait_cap_seconds, int suppress_arrive);
 
 #ifdef __cplusplus
 }

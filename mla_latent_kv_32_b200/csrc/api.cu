@@ -421,6 +421,11 @@ mla_status_t mla_decode_attention_cudacore(const mla_bf16_t *q_full, const mla_b
                       status, stream, true);
 }
 
+mla_status_t mla_debug_decode_wait(double wait_cap_seconds, int suppress_arrive) {
+  clear_error();
+  return set_decode_wait(wait_cap_seconds, suppress_arrive);
+}
+
 mla_status_t mla_out_absorb(const mla_bf16_t *o_latent, const mla_bf16_t *w_uv, int T, int n_h,
                             mla_bf16_t *u, int ld_u, mla_stream_t stream) {
   clear_error();

@@ -92,7 +92,6 @@ static_assert(kSmemBytes <= 232448, "shared memory budget");
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemO = 0;      // [0, 256): output accumulator, chunk j at 128 j
 constexpr uint32_t kTmemS = 256;    // [256, 512): two 128-column score buffers
-constexpr uint64_t kTimeoutNs = 1000000000ull;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 struct PairArgs {
@@ -105,12 +104,15 @@ struct PairArgs {
   uint16_t *o_latent;
   float *lse;
   uint32_t *status;
+  uint64_t wait_ns;     // bound of every barrier wait
+  int suppress_arrive;  // test hook: skip the first arrival on stage 0
 };
 
 struct Ctx {
   uint32_t base;
   volatile int *abort_flag;
   uint32_t *status;
+  uint64_t wait_ns;
   __device__ uint32_t bar(int i) const { return base + kOffBar + 8u * i; }
 };
 
@@ -123,11 +125,24 @@ __device__ __noinline__ bool wait_bar(const Ctx &c, uint32_t bar, uint32_t parit
     if (cluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
     if ((it & 63) == 0) {
       if (*c.abort_flag) return false;
-      if (globaltimer_ns() - t0 > kTimeoutNs) {
+      if (globaltimer_ns() - t0 > c.wait_ns) {
         *c.abort_flag = 1;
         report(c.status, MLA_DEV_TIMEOUT);
         return false;
       }
+    }
+  }
+}
+
+// Wait used to drain work this CTA issued before it leaves: ignores the abort
+// flag (the loads and MMAs in flight must land first) but keeps the time cap.
+__device__ __noinline__ bool wait_drain(const Ctx &c, uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 0;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63) == 63 && globaltimer_ns() - t0 > c.wait_ns) {
+      report(c.status, MLA_DEV_TIMEOUT);
+      return false;
     }
   }
 }
@@ -194,6 +209,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_cache,
   c.base = base;
   c.abort_flag = reinterpret_cast<volatile int *>(smem + kOffAbort);
   c.status = a.status;
+  c.wait_ns = a.wait_ns;
 
   if (threadIdx.x == 0) {
     *c.abort_flag = 0;
@@ -282,7 +298,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_cache,
           for (int ch = 0; ch < kChunksQK; ++ch, ++sg) {
             uint32_t stg;
             if (!acquire_stage(stg)) return false;
-            if (leader) {
+            if (leader && !(a.suppress_arrive && sg == 0)) {
               mbar_arrive_expect_tx(c.bar(B_FULL0 + stg), present * kBox);
               ++armed[stg];
             }
@@ -326,14 +342,17 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_cache,
       }
       // drain: the loads issued into every stage have landed before the CTA
       // leaves (the even CTA sees both CTAs' bytes on its barriers; the odd
-      // CTA sees its stages consumed)
+      // CTA sees its stages consumed). After an abort a barrier may never
+      // complete; one expired wait (>= the wait cap) is then long enough for
+      // every load in flight to have landed, so the drain stops there.
+      bool drained = true;
       if (leader) {
-        for (int s = 0; s < kStages; ++s)
-          if (armed[s]) wait_bar(c, c.bar(B_FULL0 + s), (armed[s] - 1) & 1, false);
-        if (q_armed) wait_bar(c, c.bar(B_QFULL), (q_armed - 1) & 1, false);
+        for (int s = 0; s < kStages && drained; ++s)
+          if (armed[s]) drained = wait_drain(c, c.bar(B_FULL0 + s), (armed[s] - 1) & 1);
+        if (q_armed && drained) wait_drain(c, c.bar(B_QFULL), (q_armed - 1) & 1);
       } else {
-        for (uint32_t k = sg > kStages ? sg - kStages : 0; k < sg; ++k)
-          wait_bar(c, c.bar(B_EMPTY0 + k % kStages), (k / kStages) & 1, false);
+        for (uint32_t k = sg > kStages ? sg - kStages : 0; k < sg && drained; ++k)
+          drained = wait_drain(c, c.bar(B_EMPTY0 + k % kStages), (k / kStages) & 1);
       }
     }
   } else if (warp == kMmaWarp) {
@@ -405,7 +424,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_cache,
         if (!pv(T - 1, np - kTilePages * (T - 1))) { ok = false; break; }
       }
       mma_commit_pair_leader(c.bar(B_FINAL));
-      wait_bar(c, c.bar(B_FINAL), 0, false);
+      wait_drain(c, c.bar(B_FINAL), 0);  // every MMA issued has completed
     }
   } else {
     // ------------------------------------------- softmax + epilogue warps ---
@@ -648,7 +667,19 @@ mla_status_t make_query_map(CUtensorMap *tm, const void *base, int T, int n_h) {
   return MLA_OK;
 }
 
+// failure-detection switch (mla_debug_decode_wait)
+uint64_t g_wait_ns = 1000000000ull;
+int g_suppress_arrive = 0;
+
 }  // namespace
+
+mla_status_t set_decode_wait(double seconds, int suppress_arrive) {
+  if (!(seconds > 0.0 && seconds <= 10.0))
+    return fail(MLA_ERR_INVALID_ARGUMENT, "wait cap %g s outside (0, 10]", seconds);
+  g_wait_ns = (uint64_t)(seconds * 1e9);
+  g_suppress_arrive = suppress_arrive ? 1 : 0;
+  return MLA_OK;
+}
 
 mla_status_t launch_decode_pair(const DecodeArgs &a, cudaStream_t stream) {
   const PlanHeader *ph = a.plan_host;
@@ -671,6 +702,8 @@ mla_status_t launch_decode_pair(const DecodeArgs &a, cudaStream_t stream) {
   t.o_latent = a.o_latent;
   t.lse = a.lse;
   t.status = a.status;
+  t.wait_ns = g_wait_ns;
+  t.suppress_arrive = g_suppress_arrive;
   MLA_CUDA_TRY(cudaFuncSetAttribute(decode_pair_kernel,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     (int)kSmemBytes));

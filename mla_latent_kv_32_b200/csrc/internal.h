@@ -72,6 +72,7 @@ struct DecodeArgs {
 };
 mla_status_t launch_decode_simt(const DecodeArgs &a, cudaStream_t stream);
 mla_status_t launch_decode_pair(const DecodeArgs &a, cudaStream_t stream);
+mla_status_t set_decode_wait(double seconds, int suppress_arrive);  // mla_debug_decode_wait
 mla_status_t launch_combine(const DecodeArgs &a, cudaStream_t stream);
 
 // The kernels behind each entry point (ops.cu).

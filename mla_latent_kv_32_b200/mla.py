@@ -62,6 +62,7 @@ SIGNATURES = {
     "mla_decode_plan": (_I, [_P, _I, _I, _I, _I, _I, _P, _SZ, ctypes.POINTER(mla_plan_info_t)]),
     "mla_decode_attention": (_I, [_P, _P, _I, _P, _I, _I, _I, _I, _F, _P, _P, _P, _SZ, _P, _P,
                                   _P, _P]),
+    "mla_debug_decode_wait": (_I, [ctypes.c_double, _I]),
     "mla_decode_attention_cudacore": (_I, [_P, _P, _I, _P, _I, _I, _I, _I, _F, _P, _P, _P, _SZ,
                                            _P, _P, _P, _P]),
     "mla_decode_attention_noalloc": (_I, [_P, _P, _I, _P, _I, _I, _I, _I, _F, _P, _P, _P, _P,
@@ -165,6 +166,12 @@ def mla_decode_attention(q_full, cache, num_pages, block_table, max_pages, batch
                                        _ptr(plan_dev), _ptr(workspace), workspace_bytes,
                                        _ptr(o_latent), _ptr(lse), _ptr(status),
                                        _stream(stream)), "mla_decode_attention")
+
+
+def mla_debug_decode_wait(wait_cap_seconds: float = 1.0, suppress_arrive: int = 0):
+    """Failure-detection switch of the tensor-core decode kernel (include/mla_debug.h)."""
+    _check(load().mla_debug_decode_wait(float(wait_cap_seconds), int(suppress_arrive)),
+           "mla_debug_decode_wait")
 
 
 def mla_decode_attention_cudacore(q_full, cache, num_pages, block_table, max_pages, batch, q_len,

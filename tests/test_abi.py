@@ -162,3 +162,12 @@ def test_planner_rejects_bad_input():
         mla.mla_decode_plan(np.array([5], np.int32), 1, 1, 100, 8)       # n_h 100
     buf, info = mla.mla_decode_plan(np.zeros(0, np.int32), 0, 1, 128, 8)
     assert info.num_items == 0
+
+
+def test_debug_wait_cap_validated():
+    # host-side validation of the failure-detection hook (no launch)
+    with pytest.raises(mla.MlaError):
+        mla.mla_debug_decode_wait(0.0, 0)
+    with pytest.raises(mla.MlaError):
+        mla.mla_debug_decode_wait(11.0, 0)
+    mla.mla_debug_decode_wait(1.0, 0)
