@@ -388,10 +388,11 @@ def main():
         "peak_source": f"{peak_src} (MEASURED_PEAKS.json burst figures)"
         if peak_src == "measured" else "fallback", "sources": src_hash,
     }
-    # cache_append, absorb GEMM, q RoPE pack, decode, [combine], out_absorb per
-    # timed step, plus decode [+ combine] per timed attention call
+    # cache_append, absorb GEMM (with the q RoPE pack in the same launch),
+    # decode, [combine], out_absorb per timed step, plus decode [+ combine]
+    # per timed attention call
     combine = 1 if sess.info.num_combine > 0 else 0
-    launches_timed = K * (5 + combine) + K * (1 + combine)
+    launches_timed = K * (4 + combine) + K * (1 + combine)
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": t_step, "higher_is_better": True,

@@ -149,10 +149,8 @@ mla_status_t mla_absorb_q(const mla_bf16_t *q_nope, int ld_qn, const mla_bf16_t 
   MLA_CHECK_ARG(ld_qp >= n_h * MLA_D_R && ld_qp % 8 == 0, "ld_qp too small or unaligned");
   mla_status_t st = require_sm100();
   if (st != MLA_OK) return st;
-  st = launch_absorb_q(q_nope, ld_qn, w_uk, T, n_h, q_full, (cudaStream_t)stream);
-  if (st != MLA_OK) return st;
-  return launch_q_rope_pack(q_pe, ld_qp, pos, rope_table, max_pos, T, n_h, q_full, status,
-                            (cudaStream_t)stream);
+  return launch_absorb_q(q_nope, ld_qn, q_pe, ld_qp, pos, rope_table, max_pos, w_uk, T, n_h,
+                         q_full, status, (cudaStream_t)stream);
 }
 
 size_t mla_plan_bytes(int batch, int q_len, int num_ctas) {

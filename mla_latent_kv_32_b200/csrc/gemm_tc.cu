@@ -19,8 +19,16 @@
 // are small), all four warps then read it back
 // (thread = row m) and write C through arbitrary strides, as bf16 or fp32
 // (fp32 outputs may be split over K and reduced with atomic adds).
+//
+// A launch may carry a side job in extra CTAs that run alongside the tiles:
+// the q^R RoPE/pack of mla_absorb_q (q_full[t][h][512:576] = RoPE(q^R[t][h],
+// pos[t]), interleaved pairs, fp32 table, no fused multiply-add, RNE to bf16;
+// "Deconstructing DeepSeek V4 Pro", rotational embedding), which writes
+// columns the GEMM tiles do not touch.
 #include <cuda.h>
 #include <cudaTypedefs.h>
+
+#include <algorithm>
 
 #include "internal.h"
 #include "sm100.cuh"
@@ -48,7 +56,56 @@ struct GemmTcArgs {
   long long sCz, sCm, sCn;
   int c_fp32;
   uint32_t *status;
+  int tile_z;           // z extent of the GEMM tiles; CTAs beyond it run the side job
+  // side job (rope_q_pe == nullptr: none)
+  const uint16_t *rope_q_pe;
+  int rope_ld_qp;
+  const int32_t *rope_pos;
+  const float *rope_table;
+  int rope_max_pos, rope_T, rope_n_h;
+  uint16_t *rope_q_full;
 };
+
+// Side job: each thread rotates the 4 pairs of one 16-byte chunk of q^R
+// (8 chunks per token-head), striding over all chunks.
+__device__ void rope_side_job(const GemmTcArgs &g, int cta, int ctas) {
+  const long long chunks = (long long)g.rope_T * g.rope_n_h * 8;
+  for (long long c = (long long)cta * blockDim.x + threadIdx.x; c < chunks;
+       c += (long long)ctas * blockDim.x) {
+    const int q = (int)(c & 7);
+    const long long th = c >> 3;
+    const int t = (int)(th / g.rope_n_h), h = (int)(th % g.rope_n_h);
+    const uint4 kv = __ldg(reinterpret_cast<const uint4 *>(g.rope_q_pe + (size_t)t * g.rope_ld_qp +
+                                                           h * MLA_D_R) + q);
+    uint4 *dst = reinterpret_cast<uint4 *>(g.rope_q_full + ((size_t)t * g.rope_n_h + h) * MLA_ROW +
+                                           MLA_D_C) + q;
+    if (g.rope_pos == nullptr) {
+      *dst = kv;
+      continue;
+    }
+    const int p = __ldg(g.rope_pos + t);
+    if (p < 0 || p >= g.rope_max_pos) {
+      if (q == 0) report(g.status, MLA_DEV_BAD_POSITION);
+      *dst = make_uint4(0, 0, 0, 0);
+      continue;
+    }
+    const float4 cs0 = __ldg(reinterpret_cast<const float4 *>(g.rope_table + (size_t)p * 64 + q * 8));
+    const float4 cs1 =
+        __ldg(reinterpret_cast<const float4 *>(g.rope_table + (size_t)p * 64 + q * 8 + 4));
+    const uint32_t wv[4] = {kv.x, kv.y, kv.z, kv.w};
+    const float cosv[4] = {cs0.x, cs0.z, cs1.x, cs1.z};
+    const float sinv[4] = {cs0.y, cs0.w, cs1.y, cs1.w};
+    uint32_t out[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float y0, y1;
+      rope_pair_rn(bf16_bits_to_f32(wv[i] & 0xFFFFu), bf16_bits_to_f32(wv[i] >> 16), cosv[i],
+                   sinv[i], y0, y1);
+      out[i] = pack_bf16x2(y0, y1);
+    }
+    *dst = make_uint4(out[0], out[1], out[2], out[3]);
+  }
+}
 
 __device__ __noinline__ bool wait_bar_g(uint32_t bar, uint32_t parity, uint32_t *status) {
   if (mbar_try_wait(bar, parity)) return true;
@@ -65,6 +122,13 @@ __device__ __noinline__ bool wait_bar_g(uint32_t bar, uint32_t parity, uint32_t 
 __global__ void __launch_bounds__(128, 4)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                const GemmTcArgs g) {
+  if ((int)blockIdx.z >= g.tile_z) {
+    // side-job CTAs: no shared memory, barriers or tensor memory
+    const int per_z = gridDim.x * gridDim.y;
+    const int cta = ((int)blockIdx.z - g.tile_z) * per_z + blockIdx.y * gridDim.x + blockIdx.x;
+    rope_side_job(g, cta, ((int)gridDim.z - g.tile_z) * per_z);
+    return;
+  }
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -245,6 +309,22 @@ mla_status_t launch_gemm_tc(const GemmTcDesc &d, cudaStream_t stream) {
   g.sCn = d.sCn;
   g.c_fp32 = d.c_fp32;
   g.status = d.status;
+  g.tile_z = d.batch * splits;
+  g.rope_q_pe = d.rope_q_pe;
+  g.rope_ld_qp = d.rope_ld_qp;
+  g.rope_pos = d.rope_pos;
+  g.rope_table = d.rope_table;
+  g.rope_max_pos = d.rope_max_pos;
+  g.rope_T = d.rope_T;
+  g.rope_n_h = d.rope_n_h;
+  g.rope_q_full = d.rope_q_full;
+  // side-job CTAs: whole z-slices of the grid, ~64 CTAs of 128 threads
+  int side_z = 0;
+  if (d.rope_q_pe != nullptr && d.rope_T > 0) {
+    const long long chunks = (long long)d.rope_T * d.rope_n_h * 8;
+    const long long want = std::min<long long>(64, (chunks + 127) / 128);
+    side_z = (int)((want + ntile * mtile - 1) / (ntile * mtile));
+  }
   if (splits > 1) {
     if (!d.c_contiguous)
       return fail(MLA_ERR_UNSUPPORTED, "split-K needs a contiguous fp32 output");
@@ -252,7 +332,7 @@ mla_status_t launch_gemm_tc(const GemmTcDesc &d, cudaStream_t stream) {
   }
   MLA_CUDA_TRY(cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     (int)smem_bytes));
-  dim3 grid(ntile, mtile, d.batch * splits);
+  dim3 grid(ntile, mtile, d.batch * splits + side_z);
   gemm_tc_kernel<<<grid, 128, smem_bytes, stream>>>(tm_a, tm_b, g);
   MLA_LAUNCH_CHECK("gemm_tc_kernel");
   return MLA_OK;

@@ -6,21 +6,6 @@
 
 namespace mla {
 
-// Generic strided, batched bf16 GEMM on CUDA cores (fp32 accumulation):
-//   C[z][m][n] = sum_k A[z][m][k] * B[z][n][k]
-// element (z,m,k) of A at A + z*sAz + m*sAm + k*sAk, likewise B and C.
-struct GemmArgs {
-  const uint16_t *A;
-  long long sAz, sAm, sAk;
-  const uint16_t *B;
-  long long sBz, sBn, sBk;
-  void *C;
-  long long sCz, sCm, sCn;
-  int c_fp32;
-  int M, N, K, batch;
-};
-mla_status_t launch_gemm_simt(const GemmArgs &g, cudaStream_t stream);
-
 // Tensor-core GEMM: C[z][m][n] = sum_k A[z][m][k] * B[z][n][k].
 // A element (z,m,k): K-major at A + z*sAz + m*sAm + k, or (a_mn) MN-major at
 // A + z*sAz + k*sAk + m. B element (z,n,k) at B + z*sBz + n*sBn + k.
@@ -39,13 +24,17 @@ struct GemmTcDesc {
   int c_contiguous;      // C occupies c_bytes contiguous bytes (needed for the split)
   size_t c_bytes;
   uint32_t *status;
+  // Optional side job run by extra CTAs of the same launch (concurrently with
+  // the GEMM tiles): q_full[t][h][512:576] = RoPE(q_pe[t][h][:], pos[t]) (a
+  // copy when pos == NULL). Off when rope_q_pe == NULL.
+  const uint16_t *rope_q_pe;
+  int rope_ld_qp;
+  const int32_t *rope_pos;
+  const float *rope_table;
+  int rope_max_pos, rope_T, rope_n_h;
+  uint16_t *rope_q_full;
 };
 mla_status_t launch_gemm_tc(const GemmTcDesc &d, cudaStream_t stream);
-
-// q_full[t][h][512:576] = RoPE(q_pe[t][h][:], pos[t]) (or copy when pos == NULL).
-mla_status_t launch_q_rope_pack(const uint16_t *q_pe, int ld_qp, const int32_t *pos,
-                                const float *rope_table, int max_pos, int T, int n_h,
-                                uint16_t *q_full, uint32_t *status, cudaStream_t stream);
 
 mla_status_t launch_cache_append(uint16_t *cache, int num_pages, const int32_t *block_table,
                                  int batch, int max_pages, const int32_t *seq_idx,
@@ -76,8 +65,10 @@ mla_status_t set_decode_wait(double seconds, int suppress_arrive);  // mla_debug
 mla_status_t launch_combine(const DecodeArgs &a, cudaStream_t stream);
 
 // The kernels behind each entry point (ops.cu).
-mla_status_t launch_absorb_q(const uint16_t *q_nope, int ld_qn, const uint16_t *w_uk, int T,
-                             int n_h, uint16_t *q_full, cudaStream_t stream);
+mla_status_t launch_absorb_q(const uint16_t *q_nope, int ld_qn, const uint16_t *q_pe, int ld_qp,
+                             const int32_t *pos, const float *rope_table, int max_pos,
+                             const uint16_t *w_uk, int T, int n_h, uint16_t *q_full,
+                             uint32_t *status, cudaStream_t stream);
 mla_status_t launch_out_absorb(const uint16_t *o_latent, const uint16_t *w_uv, int T, int n_h,
                                uint16_t *u, int ld_u, cudaStream_t stream);
 mla_status_t launch_projection(const uint16_t *X, int ld_x, const uint16_t *W, int ld_w, void *C,

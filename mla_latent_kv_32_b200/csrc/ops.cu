@@ -4,14 +4,20 @@
 namespace mla {
 
 // q_full[t][h][c] = sum_d q_nope[t][h][d] * w_uk[h][d][c]   (batched over heads;
-// m = latent column c, n = token t, k = d; W^UK read as its transpose)
-mla_status_t launch_absorb_q(const uint16_t *q_nope, int ld_qn, const uint16_t *w_uk, int T,
-                             int n_h, uint16_t *q_full, cudaStream_t stream) {
+// m = latent column c, n = token t, k = d; W^UK read as its transpose), and in
+// the same launch q_full[t][h][512:576] = RoPE(q_pe[t][h], pos[t])
+mla_status_t launch_absorb_q(const uint16_t *q_nope, int ld_qn, const uint16_t *q_pe, int ld_qp,
+                             const int32_t *pos, const float *rope_table, int max_pos,
+                             const uint16_t *w_uk, int T, int n_h, uint16_t *q_full,
+                             uint32_t *status, cudaStream_t stream) {
   GemmTcDesc d = {};
   d.A = w_uk; d.sAz = (long long)MLA_D_NOPE * MLA_D_C; d.sAk = MLA_D_C; d.a_mn = 1;
   d.B = q_nope; d.sBz = MLA_D_NOPE; d.sBn = ld_qn;
   d.C = q_full; d.sCz = MLA_ROW; d.sCm = 1; d.sCn = (long long)n_h * MLA_ROW;
   d.c_fp32 = 0; d.M = MLA_D_C; d.N = T; d.K = MLA_D_NOPE; d.batch = n_h;
+  d.status = status;
+  d.rope_q_pe = q_pe; d.rope_ld_qp = ld_qp; d.rope_pos = pos; d.rope_table = rope_table;
+  d.rope_max_pos = max_pos; d.rope_T = T; d.rope_n_h = n_h; d.rope_q_full = q_full;
   return launch_gemm_tc(d, stream);
 }
 
