@@ -61,6 +61,10 @@ def parse():
     ap.add_argument("--max-split", type=int, default=-1)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--rows", action="store_true",
+                    help="time every library call of the decode step (v3) and of the "
+                         "full layer (layer_v3) alone against its own roofline; one JSON "
+                         "line per call")
     return ap.parse_args()
 
 
@@ -248,6 +252,90 @@ def workload_config(w, inp, sess):
     return cfg
 
 
+def run_rows(args):
+    """Each call of the path alone, L2 flushed before every call: time, its
+    algorithmic bytes (weights and activations read once, outputs written
+    once) and FLOPs, and the fraction of the roofline (the slower of bytes ÷
+    measured HBM bandwidth and FLOPs ÷ measured bf16 peak)."""
+    import torch
+    import synth
+    from mla_latent_kv_32_b200 import build as build_mod
+    from mla_latent_kv_32_b200 import mla
+    from mla_latent_kv_32_b200.runtime import DecodeSession, LayerSession
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    build_mod.build()
+    mla.load()
+    peaks, peak_src = load_peaks()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def timed(fn, K):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(K):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b) * 1e3)
+        return statistics.median(ts)
+
+    def line(workload, row, call, us, nbytes, flops):
+        t_mem = nbytes / (peaks["hbm_gbs"] * 1e9) * 1e6
+        t_tc = flops / (peaks["bf16_tflops"] * 1e12) * 1e6
+        out = {"mode": "rows", "workload": workload, "row": row, "call": call, "us": us,
+               "bytes": int(nbytes), "flops": float(flops),
+               "gbs": nbytes / us / 1e3, "tflops": flops / us / 1e6,
+               "bound": "hbm" if t_mem >= t_tc else "tensor",
+               "roofline_us": max(t_mem, t_tc), "frac": max(t_mem, t_tc) / us,
+               "peak_source": peak_src}
+        print(json.dumps(out), flush=True)
+
+    K = max(5, args.steps)
+    bf = 2
+    # decode step rows on v3
+    w = synth.WORKLOADS["v3"]
+    inp = synth.make_decode_inputs(w)
+    sess = DecodeSession(inp, dev)
+    T, H = w.B * w.q_len, w.n_h
+    line("v3", "a3+a4", "mla_cache_append", timed(sess.append, K),
+         T * (576 * bf + 1152 + 256), 0)
+    line("v3", "a3+a5", "mla_absorb_q", timed(sess.absorb, K),
+         H * 128 * 512 * bf + T * H * (128 + 64 + 576) * bf + T * 256, 2.0 * T * H * 128 * 512)
+    cache = int(inp.lens.sum()) * ROW_BYTES
+    vis = sum(int(L) - w.q_len + j + 1 for L in inp.lens for j in range(w.q_len))
+    line("v3", "a6+a7", "mla_decode_attention", timed(sess.attend, K), cache,
+         float(vis) * H * FLOP_PER_TOKEN_HEAD)
+    line("v3", "a8", "mla_out_absorb", timed(sess.expand, K),
+         H * 128 * 512 * bf + T * H * (512 + 128) * bf, 2.0 * T * H * 128 * 512)
+    del sess, inp
+    torch.cuda.empty_cache()
+    # the whole layer's projections on layer_v3
+    w = synth.WORKLOADS["layer_v3"]
+    inp = synth.make_layer_inputs(w)
+    ls = LayerSession(inp, dev)
+    Tq, Tk, H, d, ql = ls.Tq, ls.T, w.n_h, w.hidden, w.q_lora
+    nq = H * 192
+    line("layer_v3", "a1", "mla_gemm_bf16 x2 (W_DQ, [W_UQ|W_QR])", timed(ls.project_q, K),
+         (ql * d + Tq * d + Tq * ql) * bf + (nq * ql + Tq * ql + Tq * nq) * bf,
+         2.0 * Tq * ql * d + 2.0 * Tq * nq * ql)
+    line("layer_v3", "a2", "mla_gemm_bf16 ([W_DKV|W_KR])", timed(ls.project_kv, K),
+         (576 * d + Tk * d + Tk * 576) * bf, 2.0 * Tk * 576 * d)
+    ls.project_q(); ls.project_kv(); ls.append(); ls.absorb()
+    line("layer_v3", "a6+a7", "mla_decode_attention", timed(ls.attend, K),
+         int(ls.lens.sum()) * ROW_BYTES,
+         float(sum(int(L) for L in ls.lens)) * H * FLOP_PER_TOKEN_HEAD)
+    line("layer_v3", "a9", "mla_gemm_bf16 (W_O, fp32 out)", timed(ls.project_out, K),
+         (d * H * 128 + Tq * H * 128) * bf + Tq * d * 4, 2.0 * Tq * d * H * 128)
+    return 0
+
+
 def main():
     args = parse()
     rank = int(os.environ.get("RANK", "0"))
@@ -255,6 +343,8 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         return run_reference(args, rank, world)
+    if args.rows:
+        return run_rows(args) if rank == 0 else 0
 
     import torch
     import torch.distributed as dist

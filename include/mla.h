@@ -259,6 +259,22 @@ mla_status_t mla_gemm_bf16(const mla_bf16_t *X, int ld_x, const mla_bf16_t *W, i
                            mla_stream_t stream);
 
 /*
+ * mla_gemm_bf16_ws -- device. mla_gemm_bf16 with a caller workspace for
+ * bf16 outputs: when the output has few 128 x 256 tiles and K is long (the
+ * down-projections from the 7168-wide hidden state), the reduction is split
+ * over K across more CTAs, fp32 partial sums accumulate in the workspace
+ * (zeroed by the call) and one more kernel rounds them to bf16 into C. Same
+ * result as mla_gemm_bf16 up to the order of the fp32 additions.
+ *   workspace: device, 16-byte aligned, >= mla_gemm_bf16_workspace_bytes(M,
+ *              N, K) bytes, or NULL (then exactly mla_gemm_bf16).
+ * The workspace must not be in use by another call running at the same time.
+ */
+size_t mla_gemm_bf16_workspace_bytes(int M, int N, int K);
+mla_status_t mla_gemm_bf16_ws(const mla_bf16_t *X, int ld_x, const mla_bf16_t *W, int ld_w,
+                              void *C, int ld_c, int c_fp32, int M, int N, int K,
+                              void *workspace, size_t workspace_bytes, mla_stream_t stream);
+
+/*
  * mla_read_status -- host. Synchronises `stream`, copies the device status
  * word to *bits and, if clear != 0, zeroes it. Returns MLA_ERR_DEVICE if any
  * bit was set, MLA_OK otherwise.

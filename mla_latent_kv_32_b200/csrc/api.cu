@@ -442,6 +442,17 @@ mla_status_t mla_out_absorb(const mla_bf16_t *o_latent, const mla_bf16_t *w_uv, 
 
 mla_status_t mla_gemm_bf16(const mla_bf16_t *X, int ld_x, const mla_bf16_t *W, int ld_w, void *C,
                            int ld_c, int c_fp32, int M, int N, int K, mla_stream_t stream) {
+  return mla_gemm_bf16_ws(X, ld_x, W, ld_w, C, ld_c, c_fp32, M, N, K, nullptr, 0, stream);
+}
+
+size_t mla_gemm_bf16_workspace_bytes(int M, int N, int K) {
+  if (M <= 0 || N <= 0 || K <= 0) return 0;
+  return ((size_t)M * N * sizeof(float) + 255) & ~(size_t)255;
+}
+
+mla_status_t mla_gemm_bf16_ws(const mla_bf16_t *X, int ld_x, const mla_bf16_t *W, int ld_w,
+                              void *C, int ld_c, int c_fp32, int M, int N, int K, void *workspace,
+                              size_t workspace_bytes, mla_stream_t stream) {
   clear_error();
   MLA_CHECK_ARG(M >= 0 && N >= 0 && K >= 0, "negative size");
   if (M == 0 || N == 0) return MLA_OK;
@@ -452,9 +463,14 @@ mla_status_t mla_gemm_bf16(const mla_bf16_t *X, int ld_x, const mla_bf16_t *W, i
   MLA_CHECK_ARG(aligned16(X) && aligned16(W) && aligned16(C), "pointers must be 16-byte aligned");
   MLA_CHECK_ARG(ld_x % 8 == 0 && ld_w % 8 == 0 && ld_c % (c_fp32 ? 4 : 8) == 0,
                 "leading dimensions must keep rows 16-byte aligned");
+  MLA_CHECK_ARG(workspace == nullptr || aligned16(workspace), "workspace must be 16-byte aligned");
   mla_status_t st = require_sm100();
   if (st != MLA_OK) return st;
-  return launch_projection(X, ld_x, W, ld_w, C, ld_c, c_fp32, M, N, K, (cudaStream_t)stream);
+  const bool use_ws = workspace != nullptr && !c_fp32 &&
+                      workspace_bytes >= mla_gemm_bf16_workspace_bytes(M, N, K);
+  return launch_projection(X, ld_x, W, ld_w, C, ld_c, c_fp32, M, N, K,
+                           use_ws ? static_cast<float *>(workspace) : nullptr,
+                           (cudaStream_t)stream);
 }
 
 mla_status_t mla_read_status(uint32_t *status, uint32_t *bits, int clear, mla_stream_t stream) {

@@ -55,6 +55,7 @@ struct GemmTcArgs {
   void *C;
   long long sCz, sCm, sCn;
   int c_fp32;
+  float *ws;            // bf16 output split over K: fp32 sums at ((z*N + n)*M + m)
   uint32_t *status;
   int tile_z;           // z extent of the GEMM tiles; CTAs beyond it run the side job
   // side job (rope_q_pe == nullptr: none)
@@ -214,8 +215,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__
     for (int e = 0; e < 32; ++e) {
       const int n = n0 + 32 * ch + e;
       if (n >= g.N) break;
-      const long long off = (long long)z * g.sCz + (long long)m * g.sCm + (long long)n * g.sCn;
       const float v = __uint_as_float(r[e]);
+      if (g.ws != nullptr) {
+        atomicAdd(g.ws + ((long long)z * g.N + n) * g.M + m, v);
+        continue;
+      }
+      const long long off = (long long)z * g.sCz + (long long)m * g.sCm + (long long)n * g.sCn;
       if (g.c_fp32) {
         if (g.splits > 1)
           atomicAdd(reinterpret_cast<float *>(g.C) + off, v);
@@ -231,6 +236,21 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, g.tmem_cols);
+  }
+}
+
+// C[z][m][n] (bf16, strided) = the fp32 split-K sums ws[(z*N + n)*M + m].
+__global__ void __launch_bounds__(256)
+split_to_bf16_kernel(const float *__restrict__ ws, int M, int N, int batch, uint16_t *C,
+                     long long sCz, long long sCm, long long sCn) {
+  const long long total = (long long)M * N * batch;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int m = (int)(i % M);
+    const long long zn = i / M;
+    const int n = (int)(zn % N), z = (int)(zn / N);
+    C[(long long)z * sCz + (long long)m * sCm + (long long)n * sCn] =
+        (uint16_t)f32_to_bf16_bits(ws[i]);
   }
 }
 
@@ -289,11 +309,12 @@ mla_status_t launch_gemm_tc(const GemmTcDesc &d, cudaStream_t stream) {
   const int kchunks = (d.K + 63) / 64;
   const int ntile = (d.N + BN - 1) / BN, mtile = (d.M + 127) / 128;
   int splits = 1;
-  if (d.c_fp32 && d.allow_split) {
+  if ((d.c_fp32 && d.allow_split) || (!d.c_fp32 && d.split_ws != nullptr)) {
     // spread long reductions over more CTAs when the tile grid is small
     const int ctas = ntile * mtile * d.batch;
-    while (splits < 8 && ctas * splits * 2 <= 296 && kchunks / (splits * 2) >= 4) splits *= 2;
+    while (splits < 32 && ctas * splits * 2 <= 296 && kchunks / (splits * 2) >= 4) splits *= 2;
   }
+  const bool ws_split = splits > 1 && !d.c_fp32;
   g.splits = splits;
   g.k_chunks = (kchunks + splits - 1) / splits;
   g.stages = g.k_chunks < kMaxStages ? g.k_chunks : kMaxStages;
@@ -308,6 +329,7 @@ mla_status_t launch_gemm_tc(const GemmTcDesc &d, cudaStream_t stream) {
   g.sCm = d.sCm;
   g.sCn = d.sCn;
   g.c_fp32 = d.c_fp32;
+  g.ws = ws_split ? d.split_ws : nullptr;
   g.status = d.status;
   g.tile_z = d.batch * splits;
   g.rope_q_pe = d.rope_q_pe;
@@ -325,7 +347,10 @@ mla_status_t launch_gemm_tc(const GemmTcDesc &d, cudaStream_t stream) {
     const long long want = std::min<long long>(64, (chunks + 127) / 128);
     side_z = (int)((want + ntile * mtile - 1) / (ntile * mtile));
   }
-  if (splits > 1) {
+  if (ws_split) {
+    MLA_CUDA_TRY(cudaMemsetAsync(d.split_ws, 0, (size_t)d.M * d.N * d.batch * sizeof(float),
+                                 stream));
+  } else if (splits > 1) {
     if (!d.c_contiguous)
       return fail(MLA_ERR_UNSUPPORTED, "split-K needs a contiguous fp32 output");
     MLA_CUDA_TRY(cudaMemsetAsync(d.C, 0, d.c_bytes, stream));
@@ -335,6 +360,14 @@ mla_status_t launch_gemm_tc(const GemmTcDesc &d, cudaStream_t stream) {
   dim3 grid(ntile, mtile, d.batch * splits + side_z);
   gemm_tc_kernel<<<grid, 128, smem_bytes, stream>>>(tm_a, tm_b, g);
   MLA_LAUNCH_CHECK("gemm_tc_kernel");
+  if (ws_split) {
+    const long long total = (long long)d.M * d.N * d.batch;
+    const int blocks = (int)std::min<long long>(1184, (total + 255) / 256);
+    split_to_bf16_kernel<<<blocks, 256, 0, stream>>>(d.split_ws, d.M, d.N, d.batch,
+                                                      static_cast<uint16_t *>(d.C), d.sCz, d.sCm,
+                                                      d.sCn);
+    MLA_LAUNCH_CHECK("split_to_bf16_kernel");
+  }
   return MLA_OK;
 }
 

@@ -24,6 +24,10 @@ struct GemmTcDesc {
   int c_contiguous;      // C occupies c_bytes contiguous bytes (needed for the split)
   size_t c_bytes;
   uint32_t *status;
+  // bf16 output with a split over K: fp32 partial sums accumulate in
+  // split_ws (M*N*batch floats, element (z, n, m) at (z*N + n)*M + m), then
+  // are rounded into C. NULL: bf16 outputs are never split.
+  float *split_ws;
   // Optional side job run by extra CTAs of the same launch (concurrently with
   // the GEMM tiles): q_full[t][h][512:576] = RoPE(q_pe[t][h][:], pos[t]) (a
   // copy when pos == NULL). Off when rope_q_pe == NULL.
@@ -72,7 +76,8 @@ mla_status_t launch_absorb_q(const uint16_t *q_nope, int ld_qn, const uint16_t *
 mla_status_t launch_out_absorb(const uint16_t *o_latent, const uint16_t *w_uv, int T, int n_h,
                                uint16_t *u, int ld_u, cudaStream_t stream);
 mla_status_t launch_projection(const uint16_t *X, int ld_x, const uint16_t *W, int ld_w, void *C,
-                               int ld_c, int c_fp32, int M, int N, int K, cudaStream_t stream);
+                               int ld_c, int c_fp32, int M, int N, int K, float *split_ws,
+                               cudaStream_t stream);
 mla_status_t launch_decode(const DecodeArgs &a, cudaStream_t stream);
 
 }  // namespace mla

@@ -35,7 +35,8 @@ mla_status_t launch_out_absorb(const uint16_t *o_latent, const uint16_t *w_uv, i
 
 // C[t][f] = sum_k X[t][k] * W[f][k]   (m = output feature f, n = token t)
 mla_status_t launch_projection(const uint16_t *X, int ld_x, const uint16_t *W, int ld_w, void *C,
-                               int ld_c, int c_fp32, int M, int N, int K, cudaStream_t stream) {
+                               int ld_c, int c_fp32, int M, int N, int K, float *split_ws,
+                               cudaStream_t stream) {
   GemmTcDesc d = {};
   d.A = W; d.sAz = 0; d.sAm = ld_w; d.a_mn = 0;
   d.B = X; d.sBz = 0; d.sBn = ld_x;
@@ -44,6 +45,7 @@ mla_status_t launch_projection(const uint16_t *X, int ld_x, const uint16_t *W, i
   d.allow_split = c_fp32;
   d.c_contiguous = 1;
   d.c_bytes = (size_t)M * ld_c * (c_fp32 ? 4 : 2);
+  d.split_ws = c_fp32 ? nullptr : split_ws;
   return launch_gemm_tc(d, stream);
 }
 

@@ -69,6 +69,8 @@ SIGNATURES = {
                                           _P, _P]),
     "mla_out_absorb": (_I, [_P, _P, _I, _I, _P, _I, _P]),
     "mla_gemm_bf16": (_I, [_P, _I, _P, _I, _P, _I, _I, _I, _I, _I, _P]),
+    "mla_gemm_bf16_workspace_bytes": (_SZ, [_I, _I, _I]),
+    "mla_gemm_bf16_ws": (_I, [_P, _I, _P, _I, _P, _I, _I, _I, _I, _I, _P, _SZ, _P]),
     "mla_read_status": (_I, [_P, _P, _I, _P]),
 }
 
@@ -204,6 +206,17 @@ def mla_out_absorb(o_latent, w_uv, T, n_h, u, ld_u, stream=None):
 def mla_gemm_bf16(X, ld_x, W, ld_w, C, ld_c, c_fp32, M, N, K, stream=None):
     _check(load().mla_gemm_bf16(_ptr(X), ld_x, _ptr(W), ld_w, _ptr(C), ld_c, int(c_fp32), M, N,
                                 K, _stream(stream)), "mla_gemm_bf16")
+
+
+def mla_gemm_bf16_workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(load().mla_gemm_bf16_workspace_bytes(M, N, K))
+
+
+def mla_gemm_bf16_ws(X, ld_x, W, ld_w, C, ld_c, c_fp32, M, N, K, workspace, workspace_bytes,
+                     stream=None):
+    _check(load().mla_gemm_bf16_ws(_ptr(X), ld_x, _ptr(W), ld_w, _ptr(C), ld_c, int(c_fp32), M,
+                                   N, K, _ptr(workspace), int(workspace_bytes), _stream(stream)),
+           "mla_gemm_bf16_ws")
 
 
 def mla_read_status(status, clear: bool = True, stream=None) -> int:

@@ -260,34 +260,74 @@ class LayerSession:
         self.lse = torch.empty((self.Tq, self.n_h), dtype=torch.float32, device=dev)
         self.u = torch.empty((self.Tq, self.n_h * D_V), dtype=torch.bfloat16, device=dev)
         self.out = torch.empty((self.Tq, self.hidden), dtype=torch.float32, device=dev)
+        self.gemm_ws = None
+        self._gemm_ws()   # allocated here, not during a step
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
 
-    def step(self, stream=None):
+    # the layer's calls one by one (step runs them in this order) -------------
+    def _gemm_ws(self):
+        # split-K workspace of the two down-projections from the hidden state
+        if getattr(self, "gemm_ws", None) is None:
+            need = max(mla.mla_gemm_bf16_workspace_bytes(self.Tq, max(self.q_lora, 1), self.hidden),
+                       mla.mla_gemm_bf16_workspace_bytes(self.T, ROW, self.hidden))
+            self.gemm_ws = torch.empty(max(need, 256), dtype=torch.uint8, device=self.device)
+        return self.gemm_ws
+
+    def project_q(self, stream=None):
         n_h, d = self.n_h, self.hidden
         hq = self.h[self.T - self.Tq:]
         nq = n_h * (D_NOPE + D_R)
         if self.q_lora:
-            mla.mla_gemm_bf16(hq, d, self.w_dq, d, self.cq, self.q_lora, 0, self.Tq, self.q_lora,
-                              d, stream)
+            ws = self._gemm_ws()
+            mla.mla_gemm_bf16_ws(hq, d, self.w_dq, d, self.cq, self.q_lora, 0, self.Tq,
+                                 self.q_lora, d, ws, ws.numel(), stream)
             mla.mla_gemm_bf16(self.cq, self.q_lora, self.w_qcat, self.q_lora, self.q, nq, 0,
                               self.Tq, nq, self.q_lora, stream)
         else:
             mla.mla_gemm_bf16(hq, d, self.w_qcat, d, self.q, nq, 0, self.Tq, nq, d, stream)
-        mla.mla_gemm_bf16(self.h, d, self.w_kvcat, d, self.kv, ROW, 0, self.T, ROW, d, stream)
+
+    def project_kv(self, stream=None):
+        d = self.hidden
+        ws = self._gemm_ws()
+        mla.mla_gemm_bf16_ws(self.h, d, self.w_kvcat, d, self.kv, ROW, 0, self.T, ROW, d, ws,
+                             ws.numel(), stream)
+
+    def append(self, stream=None):
         kv_pe = self.kv[:, D_C:]
         mla.mla_cache_append(self.cache, self.num_pages, self.table, self.B, self.max_pages,
                              self.tok_seq, self.tok_pos, self.kv, ROW, kv_pe, ROW, self.rope,
                              self.max_pos, self.T, self.status, stream)
+
+    def absorb(self, stream=None):
+        n_h = self.n_h
+        nq = n_h * (D_NOPE + D_R)
         q_pe = self.q[:, n_h * D_NOPE:]
         mla.mla_absorb_q(self.q, nq, q_pe, nq, self.w_uk, self.q_pos, self.rope, self.max_pos,
                          self.Tq, n_h, self.q_full, self.status, stream)
+
+    def attend(self, stream=None):
         mla.mla_decode_attention(self.q_full, self.cache, self.num_pages, self.table,
-                                 self.max_pages, self.B, self.q_len, n_h, self.scale,
+                                 self.max_pages, self.B, self.q_len, self.n_h, self.scale,
                                  self.plan_host, self.plan_dev, self.workspace, self.ws_bytes,
                                  self.o, self.lse, self.status, stream)
+
+    def expand(self, stream=None):
+        n_h = self.n_h
         mla.mla_out_absorb(self.o, self.w_uv, self.Tq, n_h, self.u, n_h * D_V, stream)
+
+    def project_out(self, stream=None):
+        n_h, d = self.n_h, self.hidden
         mla.mla_gemm_bf16(self.u, n_h * D_V, self.w_o, n_h * D_V, self.out, d, 1, self.Tq, d,
                           n_h * D_V, stream)
+
+    def step(self, stream=None):
+        self.project_q(stream)
+        self.project_kv(stream)
+        self.append(stream)
+        self.absorb(stream)
+        self.attend(stream)
+        self.expand(stream)
+        self.project_out(stream)
 
     def read_status(self) -> int:
         return mla.mla_read_status(self.status, clear=True)

@@ -50,3 +50,24 @@ def test_layer(dev, name):
     got = np.stack([pool[inp.table[inp.tok_seq[t], inp.tok_pos[t] // 64], inp.tok_pos[t] % 64]
                     for t in ref["new_tok"]])
     assert_parity(O.bf16_to_f64(got), O.bf16_to_f64(ref["new_rows"]), "appended rows")
+
+
+@pytest.mark.parametrize("M,N,K", [(256, 576, 7168), (256, 1536, 7168), (7, 64, 512)])
+def test_split_k_gemm_matches_fp32(dev, M, N, K):
+    # C = X W^T with a workspace (split over K for the long reductions) against
+    # a float64 product of the same bf16 inputs; bf16 output
+    g = torch.Generator().manual_seed(M * 7 + N)
+    X = (torch.randn(M, K, generator=g) / math.sqrt(K)).to(torch.bfloat16)
+    W = torch.randn(N, K, generator=g).to(torch.bfloat16)
+    ref = (X.double() @ W.double().T).numpy()
+    Xd, Wd = X.to(dev), W.to(dev)
+    C = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(mla.mla_gemm_bf16_workspace_bytes(M, N, K), dtype=torch.uint8, device=dev)
+    mla.mla_gemm_bf16_ws(Xd, K, Wd, K, C, N, 0, M, N, K, ws, ws.numel())
+    got = C.float().cpu().numpy()
+    C2 = torch.empty_like(C)
+    mla.mla_gemm_bf16(Xd, K, Wd, K, C2, N, 0, M, N, K)
+    got2 = C2.float().cpu().numpy()
+    for g_ in (got, got2):
+        err = np.abs(g_ - ref)
+        assert err.max() <= 2e-2 * np.abs(ref).max() and err.sum() <= 5e-3 * np.abs(ref).sum()
