@@ -46,7 +46,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # decode sources it was measured on and the workload; reported only while the
 # sources match (the combine kernel's few MB are not included).
 TRAFFIC = {
-    ("e3c8d0931702c06a", "v3"): 317871616,   # decode_pair_kernel
+    ("376d5e91cc46aef1", "v3"): 318149120,   # decode_pair_kernel
 }
 
 
