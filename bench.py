@@ -208,7 +208,8 @@ def run_reference(args, rank, world):
     cores = cpu_threads()
     out = {
         "impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": None,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * w.B * w.q_len / v,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": workload_config(w, inp, None),
         "cpu_baseline": {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
@@ -241,12 +242,12 @@ def workload_config(w, inp, sess):
                        f"n_h {w.n_h}, d_c 512, d_R 64, paged cache of 64-token pages",
            "batch": w.B, "q_len": w.q_len, "n_h": w.n_h,
            "context_tokens": int(inp.lens.sum()),
-           "cache_bytes": int(inp.lens.sum()) * ROW_BYTES,
-           "l2": "flushed before every timed step and every timed attention call "
-                 "(256 MiB write, outside the events)",
-           "timing": "each step one CUDA graph replay of the four library calls; the "
-                     "attention call timed alone in a second loop for the roofline"}
+           "cache_bytes": int(inp.lens.sum()) * ROW_BYTES}
     if sess is not None:
+        cfg["l2"] = ("flushed before every timed step and every timed attention call "
+                     "(256 MiB write, outside the events)")
+        cfg["timing"] = ("each step one CUDA graph replay of the four library calls; the "
+                         "attention call timed alone in a second loop for the roofline")
         cfg["plan"] = {"work_lists": int(sess.info.num_ctas), "items": int(sess.info.num_items),
                        "partials": int(sess.info.num_partials)}
     return cfg
