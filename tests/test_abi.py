@@ -61,6 +61,23 @@ def test_invalid_arguments_rejected_before_launch(lib):
     mla.mla_out_absorb(None, None, 0, 128, None, 16384, stream=0)
 
 
+def test_empty_inputs_are_noops_without_a_device(lib):
+    """Every entry point treats an empty problem (no sequences, tokens or rows)
+    as a successful no-op that touches neither the GPU nor its pointers."""
+    for q_len in (1, 2):
+        plan, info = mla.mla_decode_plan(np.zeros(0, np.int32), 0, q_len, 128, num_ctas=8)
+        assert info.num_items == 0 and info.num_partials == 0 and info.workspace_bytes == 0
+        for fn in (mla.mla_decode_attention, mla.mla_decode_attention_cudacore):
+            fn(None, None, 1, None, 1, 0, q_len, 128, 0.07, plan, plan, None, 0, None, stream=0)
+        mla.mla_decode_attention_noalloc(None, None, 1, None, 1, 0, q_len, 128, 0.07, plan, plan,
+                                         None, stream=0)
+    mla.mla_absorb_q(None, 16384, None, 8192, None, None, None, 0, 0, 128, None, stream=0)
+    mla.mla_gemm_bf16(None, 64, None, 64, None, 64, 0, 0, 64, 64, stream=0)      # M = 0
+    mla.mla_gemm_bf16(None, 64, None, 64, None, 64, 1, 64, 0, 64, stream=0)      # N = 0
+    mla.mla_gemm_bf16_ws(None, 64, None, 64, None, 64, 0, 0, 64, 64, None, 0, stream=0)
+    assert mla.mla_gemm_bf16_workspace_bytes(0, 64, 64) == 0
+
+
 def test_rope_table_matches_oracle(lib):
     got = mla.mla_rope_table(140000)
     want = O.rope_table(140000)

@@ -92,6 +92,12 @@ SMALL = [
     ("heads32", [5000, 3, 700], 1, 32),
     ("one", [1], 1, 128),
     ("mtp_min", [2, 3], 2, 64),
+    # head counts that leave part of a CTA's 64 query rows (or all of the
+    # second CTA's) empty
+    ("heads48", [300, 64, 1], 1, 48),
+    ("heads80_mtp", [130, 2, 513], 2, 80),
+    ("heads96", [65, 4100], 1, 96),
+    ("heads112_mtp", [257, 66], 2, 112),
 ]
 
 
