@@ -38,7 +38,9 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kMaxStages = 4;
+constexpr int kMaxStages = 8;          // ring depth when one CTA per SM covers the grid
+constexpr int kSharedStages = 4;       // ring depth when CTAs share SMs
+constexpr uint32_t kSmemLimit = 232448;  // dynamic shared memory per CTA (227 KB)
 constexpr uint32_t kAStage = 128 * 128;        // 128 rows x 64 k (bf16) = 16 KB
 constexpr uint64_t kTimeoutNs = 1000000000ull;
 
@@ -68,43 +70,69 @@ struct GemmTcArgs {
 };
 
 // Side job: each thread rotates the 4 pairs of one 16-byte chunk of q^R
-// (8 chunks per token-head), striding over all chunks.
+// (8 chunks per token-head), kSideBatch chunks per pass at a stride of all
+// side threads. A pass issues every load of its chunks (values, positions)
+// before the table loads that depend on them, so a thread waits two memory
+// round trips per pass, not two per chunk.
+constexpr int kSideBatch = 4;
+
 __device__ void rope_side_job(const GemmTcArgs &g, int cta, int ctas) {
   const long long chunks = (long long)g.rope_T * g.rope_n_h * 8;
-  for (long long c = (long long)cta * blockDim.x + threadIdx.x; c < chunks;
-       c += (long long)ctas * blockDim.x) {
-    const int q = (int)(c & 7);
-    const long long th = c >> 3;
-    const int t = (int)(th / g.rope_n_h), h = (int)(th % g.rope_n_h);
-    const uint4 kv = __ldg(reinterpret_cast<const uint4 *>(g.rope_q_pe + (size_t)t * g.rope_ld_qp +
-                                                           h * MLA_D_R) + q);
-    uint4 *dst = reinterpret_cast<uint4 *>(g.rope_q_full + ((size_t)t * g.rope_n_h + h) * MLA_ROW +
-                                           MLA_D_C) + q;
-    if (g.rope_pos == nullptr) {
-      *dst = kv;
-      continue;
-    }
-    const int p = __ldg(g.rope_pos + t);
-    if (p < 0 || p >= g.rope_max_pos) {
-      if (q == 0) report(g.status, MLA_DEV_BAD_POSITION);
-      *dst = make_uint4(0, 0, 0, 0);
-      continue;
-    }
-    const float4 cs0 = __ldg(reinterpret_cast<const float4 *>(g.rope_table + (size_t)p * 64 + q * 8));
-    const float4 cs1 =
-        __ldg(reinterpret_cast<const float4 *>(g.rope_table + (size_t)p * 64 + q * 8 + 4));
-    const uint32_t wv[4] = {kv.x, kv.y, kv.z, kv.w};
-    const float cosv[4] = {cs0.x, cs0.z, cs1.x, cs1.z};
-    const float sinv[4] = {cs0.y, cs0.w, cs1.y, cs1.w};
-    uint32_t out[4];
+  const long long stride = (long long)ctas * blockDim.x;
+  for (long long c0 = (long long)cta * blockDim.x + threadIdx.x; c0 < chunks;
+       c0 += kSideBatch * stride) {
+    uint4 kv[kSideBatch];
+    int p[kSideBatch];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      float y0, y1;
-      rope_pair_rn(bf16_bits_to_f32(wv[i] & 0xFFFFu), bf16_bits_to_f32(wv[i] >> 16), cosv[i],
-                   sinv[i], y0, y1);
-      out[i] = pack_bf16x2(y0, y1);
+    for (int u = 0; u < kSideBatch; ++u) {
+      const long long c = c0 + u * stride;
+      p[u] = -1;
+      if (c >= chunks) continue;
+      const long long th = c >> 3;
+      const int t = (int)(th / g.rope_n_h), h = (int)(th % g.rope_n_h);
+      kv[u] = __ldg(reinterpret_cast<const uint4 *>(g.rope_q_pe + (size_t)t * g.rope_ld_qp +
+                                                    h * MLA_D_R) + (c & 7));
+      if (g.rope_pos != nullptr) p[u] = __ldg(g.rope_pos + t);
     }
-    *dst = make_uint4(out[0], out[1], out[2], out[3]);
+    float4 cs0[kSideBatch], cs1[kSideBatch];
+#pragma unroll
+    for (int u = 0; u < kSideBatch; ++u) {
+      const long long c = c0 + u * stride;
+      if (c >= chunks || g.rope_pos == nullptr || p[u] < 0 || p[u] >= g.rope_max_pos) continue;
+      const float *row = g.rope_table + (size_t)p[u] * 64 + (c & 7) * 8;
+      cs0[u] = __ldg(reinterpret_cast<const float4 *>(row));
+      cs1[u] = __ldg(reinterpret_cast<const float4 *>(row + 4));
+    }
+#pragma unroll
+    for (int u = 0; u < kSideBatch; ++u) {
+      const long long c = c0 + u * stride;
+      if (c >= chunks) continue;
+      const long long th = c >> 3;
+      const int t = (int)(th / g.rope_n_h), h = (int)(th % g.rope_n_h);
+      uint4 *dst = reinterpret_cast<uint4 *>(g.rope_q_full + ((size_t)t * g.rope_n_h + h) *
+                                                                 MLA_ROW + MLA_D_C) + (c & 7);
+      if (g.rope_pos == nullptr) {
+        *dst = kv[u];
+        continue;
+      }
+      if (p[u] < 0 || p[u] >= g.rope_max_pos) {
+        if ((c & 7) == 0) report(g.status, MLA_DEV_BAD_POSITION);
+        *dst = make_uint4(0, 0, 0, 0);
+        continue;
+      }
+      const uint32_t wv[4] = {kv[u].x, kv[u].y, kv[u].z, kv[u].w};
+      const float cosv[4] = {cs0[u].x, cs0[u].z, cs1[u].x, cs1[u].z};
+      const float sinv[4] = {cs0[u].y, cs0[u].w, cs1[u].y, cs1[u].w};
+      uint32_t out[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        float y0, y1;
+        rope_pair_rn(bf16_bits_to_f32(wv[i] & 0xFFFFu), bf16_bits_to_f32(wv[i] >> 16), cosv[i],
+                     sinv[i], y0, y1);
+        out[i] = pack_bf16x2(y0, y1);
+      }
+      *dst = make_uint4(out[0], out[1], out[2], out[3]);
+    }
   }
 }
 
@@ -317,11 +345,22 @@ mla_status_t launch_gemm_tc(const GemmTcDesc &d, cudaStream_t stream) {
   const bool ws_split = splits > 1 && !d.c_fp32;
   g.splits = splits;
   g.k_chunks = (kchunks + splits - 1) / splits;
-  g.stages = g.k_chunks < kMaxStages ? g.k_chunks : kMaxStages;
   g.stage_bytes = kAStage + (((uint32_t)BN * 128 + 1023u) & ~1023u);
+  // A grid that fits one CTA per SM keeps every k-chunk of a tile in flight
+  // (up to kMaxStages, within the shared memory), so a tile waits one load
+  // round trip rather than one per ring cycle; denser grids keep a shallower
+  // ring and several CTAs per SM.
+  int sms = 0;
+  st = device_info(&sms, nullptr, nullptr);
+  if (st != MLA_OK) return st;
+  const uint32_t bar_bytes = 8 * (2 * kMaxStages + 2);
+  const int fit = (int)((kSmemLimit - 1024 - bar_bytes) / g.stage_bytes);
+  const long long tile_ctas = (long long)ntile * mtile * d.batch * splits;
+  const int depth = tile_ctas <= sms ? std::min(kMaxStages, fit) : kSharedStages;
+  g.stages = std::min(g.k_chunks, depth);
   g.tmem_cols = 32;
   while (g.tmem_cols < (uint32_t)BN) g.tmem_cols *= 2;
-  const uint32_t smem_bytes = g.stages * g.stage_bytes + 8 * (2 * kMaxStages + 2) + 1024;
+  const uint32_t smem_bytes = g.stages * g.stage_bytes + bar_bytes + 1024;
   g.batch = d.batch;
   g.a_mn = d.a_mn;
   g.C = d.C;
