@@ -40,6 +40,15 @@ UNIT = "tokens/s"
 ROW_BYTES = 1152                 # 576 bf16 per cached token
 FLOP_PER_TOKEN_HEAD = 2 * 576 + 2 * 512
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# B200 data-sheet figures (dense bf16), reported beside the measured peaks
+SPEC_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
+
+
+def dist_stats(xs):
+    """median / min / p90 of a list of per-call times (ms)."""
+    ys = sorted(xs)
+    p90 = ys[min(len(ys) - 1, int(math.ceil(0.9 * len(ys))) - 1)]
+    return {"median": statistics.median(ys), "min": ys[0], "p90": p90}
 
 # DRAM traffic per launch of mla_decode_attention measured by ncu
 # (dram__bytes_read.sum + dram__bytes_write.sum), keyed by the SHA-256 of the
@@ -494,6 +503,10 @@ def main():
                    "frac": tfs / peaks["bf16_tflops"]},
         "roofline_us": max(t_mem, t_tc) * 1e6, "measured_us": t_attn * 1e3,
         "frac_of_roofline": max(t_mem, t_tc) / (t_attn / 1e3),
+        "spec": {"hbm_gbs": SPEC_PEAKS["hbm_gbs"], "bf16_tflops": SPEC_PEAKS["bf16_tflops"],
+                 "frac_of_roofline": max(cache_bytes / (SPEC_PEAKS["hbm_gbs"] * 1e9),
+                                         flops / (SPEC_PEAKS["bf16_tflops"] * 1e12))
+                 / (t_attn / 1e3)},
         "peak_source": f"{peak_src} (MEASURED_PEAKS.json burst figures)"
         if peak_src == "measured" else "fallback", "sources": src_hash,
     }
@@ -509,6 +522,7 @@ def main():
         "config": workload_config(w, inp, sess),
         "cache_gbs": cache_bytes / (t_step / 1e3) / 1e9 * world,
         "attention_ms": t_attn,
+        "step_ms_stats": dist_stats(step_ms), "attention_ms_stats": dist_stats(attn_ms),
         "roofline": roof,
         "e2e": e2e,
         "gpu_launches": launches_timed,
