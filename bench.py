@@ -97,23 +97,29 @@ def decode_sources_hash():
 
 
 class ClockSampler:
-    """Samples nvidia-smi SM clocks and throttle reasons while running."""
+    """Samples nvidia-smi SM clocks and throttle reasons every 20 ms while
+    running. ``mark_start``/``mark_end`` bound the window the summary covers
+    (the clock ramp and the timed loops); samples whose active reasons include
+    GPU idle are left out, so the median is the clock under load."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    IDLE = 0x1
 
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
-        self.lines = []
+        self.lines = []        # (host time, line)
         self.thread = None
+        self.t0 = None
+        self.t1 = None
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
@@ -124,10 +130,17 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.monotonic(), line.strip()))
+
+    def mark_start(self):
+        self.t0 = time.monotonic()
+
+    def mark_end(self):
+        self.t1 = time.monotonic()
 
     def __exit__(self, *a):
         if self.proc is not None:
+            time.sleep(0.05)
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
@@ -139,26 +152,53 @@ class ClockSampler:
     def summary(self):
         if not self.lines:
             return None
-        mhz, max_mhz, reasons, power = [], 0.0, set(), []
+        mhz, max_mhz, reasons, power, idle = [], 0.0, set(), [], 0
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        lo = self.t0 if self.t0 is not None else -math.inf
+        hi = self.t1 if self.t1 is not None else math.inf
+        for t, ln in self.lines:
+            if t < lo or t > hi:
+                continue
             parts = [p.strip() for p in ln.split(",")]
             if len(parts) < 9:
                 continue
             try:
-                mhz.append(float(parts[1]))
-                max_mhz = max(max_mhz, float(parts[2]))
-                power.append(float(parts[3]))
+                active = int(parts[4], 16)
+                m, mx, pw = float(parts[1]), float(parts[2]), float(parts[3])
             except ValueError:
                 continue
+            max_mhz = max(max_mhz, mx)
+            if active & self.IDLE:
+                idle += 1
+                continue
+            mhz.append(m)
+            power.append(pw)
             for n, v in zip(names, parts[5:9]):
                 if v.lower().startswith("active"):
                     reasons.add(n)
         if not mhz:
-            return None
+            return {"sm_mhz": None, "sm_max_mhz": max_mhz or None, "reasons": [],
+                    "samples": 0, "idle_samples": idle,
+                    "note": "no nvidia-smi sample under load in the window"}
         return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": max_mhz,
-                "reasons": sorted(reasons), "samples": len(mhz),
-                "power_w_max": max(power) if power else None}
+                "reasons": sorted(reasons), "samples": len(mhz), "idle_samples": idle,
+                "power_w_max": max(power) if power else None,
+                "window": "clock ramp + timed loops, 20 ms samples, GPU-idle samples dropped"}
+
+
+def ramp_clocks(fn, seconds=0.3, sync_every=16):
+    """Runs fn() back to back for ~seconds (synchronising every sync_every
+    calls) so that the GPU's clocks reach their loaded steady state before
+    anything is timed; from idle they take a few ms to climb."""
+    import torch
+    t_end = time.monotonic() + seconds
+    n = 0
+    while time.monotonic() < t_end:
+        for _ in range(sync_every):
+            fn()
+        torch.cuda.synchronize()
+        n += sync_every
+    return n
 
 
 def cpu_threads():
@@ -257,7 +297,9 @@ def workload_config(w, inp, sess):
                      "outside the events: a 256 MiB write, then a 256 MiB read of another "
                      "buffer so that no dirty lines of the flush remain in L2")
         cfg["timing"] = ("each step one CUDA graph replay of the four library calls; the "
-                         "attention call timed alone in a second loop for the roofline")
+                         "attention call timed alone in a second loop for the roofline; "
+                         "before timing, flush + step run back to back for 0.3 s so the "
+                         "clocks reach their loaded steady state")
         cfg["plan"] = {"work_lists": int(sess.info.num_ctas), "items": int(sess.info.num_items),
                        "partials": int(sess.info.num_partials)}
     return cfg
@@ -302,7 +344,7 @@ def run_rows(args):
     def timed(fn, K):
         for _ in range(3):
             fn()
-        torch.cuda.synchronize()
+        ramp_clocks(lambda: (flush(), fn()), seconds=0.2)
         ts = []
         for _ in range(K):
             flush()
@@ -424,6 +466,8 @@ def main():
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
     ea = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
     with ClockSampler(local) as clocks:
+        clocks.mark_start()
+        ramp_clocks(lambda: (flush(), sess.replay(stream)))
         barrier()
         for k in range(K):
             flush()
@@ -436,6 +480,7 @@ def main():
             sess.attend()
             ea[k][1].record(stream)
         barrier()
+        clocks.mark_end()
     bits = sess.read_status()
     assert bits == 0, f"device status 0x{bits:x} in the timed steps"
     step_ms = [a.elapsed_time(b) for a, b in ev]
