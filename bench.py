@@ -70,6 +70,9 @@ def parse():
     ap.add_argument("--max-split", type=int, default=-1)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--ramp-seconds", type=float, default=0.3,
+                    help="back-to-back untimed steps before timing, so the clocks leave "
+                         "their idle state (0: none, e.g. under a profiler)")
     ap.add_argument("--rows", action="store_true",
                     help="time every library call of the decode step (v3) and of the "
                          "full layer (layer_v3) alone against its own roofline; one JSON "
@@ -285,7 +288,7 @@ def whole_job_rate(world, units_per_rank, t_ms):
     return world * units_per_rank / (t_ms / 1e3)
 
 
-def workload_config(w, inp, sess):
+def workload_config(w, inp, sess, ramp_seconds=0.0):
     cfg = {"workload": f"{w.name}: absorbed MLA decode, batch {w.B}, {w.q_len} query token(s) "
                        f"per sequence, context {'U[1,%d]' % w.L if w.lens == 'ragged' else w.L}, "
                        f"n_h {w.n_h}, d_c 512, d_R 64, paged cache of 64-token pages",
@@ -298,8 +301,9 @@ def workload_config(w, inp, sess):
                      "buffer so that no dirty lines of the flush remain in L2")
         cfg["timing"] = ("each step one CUDA graph replay of the four library calls; the "
                          "attention call timed alone in a second loop for the roofline; "
-                         "before timing, flush + step run back to back for 0.3 s so the "
-                         "clocks reach their loaded steady state")
+                         f"before timing, flush + step run back to back for "
+                         f"{ramp_seconds:g} s so the clocks reach their loaded steady "
+                         f"state")
         cfg["plan"] = {"work_lists": int(sess.info.num_ctas), "items": int(sess.info.num_items),
                        "partials": int(sess.info.num_partials)}
     return cfg
@@ -315,7 +319,9 @@ class L2Flush:
     def __init__(self, dev):
         import torch
         self.w = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-        self.r = torch.ones(64 << 20, dtype=torch.int32, device=dev)
+        # float32: the sum reduces the buffer in place (an int32 sum would
+        # first write a 512 MB int64 copy of it)
+        self.r = torch.ones(64 << 20, dtype=torch.float32, device=dev)
 
     def __call__(self):
         self.w.zero_()
@@ -344,7 +350,8 @@ def run_rows(args):
     def timed(fn, K):
         for _ in range(3):
             fn()
-        ramp_clocks(lambda: (flush(), fn()), seconds=0.2)
+        if args.ramp_seconds > 0:
+            ramp_clocks(lambda: (flush(), fn()), seconds=min(0.2, args.ramp_seconds))
         ts = []
         for _ in range(K):
             flush()
@@ -467,7 +474,8 @@ def main():
     ea = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
     with ClockSampler(local) as clocks:
         clocks.mark_start()
-        ramp_clocks(lambda: (flush(), sess.replay(stream)))
+        if args.ramp_seconds > 0:
+            ramp_clocks(lambda: (flush(), sess.replay(stream)), seconds=args.ramp_seconds)
         barrier()
         for k in range(K):
             flush()
@@ -564,7 +572,7 @@ def main():
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": t_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": workload_config(w, inp, sess),
+        "config": workload_config(w, inp, sess, args.ramp_seconds),
         "cache_gbs": cache_bytes / (t_step / 1e3) / 1e9 * world,
         "attention_ms": t_attn,
         "step_ms_stats": dist_stats(step_ms), "attention_ms_stats": dist_stats(attn_ms),
