@@ -25,6 +25,9 @@ What it computes, and where the pages define it:
   q^R_i . k^R_j``; ``o_i = sum_j a_j c_j``; ``u_i = W^UV_i o_i`` --
   "DeepSeek-V3 MLA ... Guide", section "Inference Optimization: The Matrix
   Absorption Trick", parts 2 and 3, and "Step 3" (``forward_decode_absorbed``).
+* Split-KV merge of partial results (``merge_partials``): the log-sum-exp
+  identity; the pages have no split, so this is the plain reading of a
+  combine that is exact in real arithmetic.
 * Whole decode layer (query compression c^Q = W^DQ h, q^C = W^UQ c^Q,
   q^R = RoPE(W^QR c^Q); c^KV = W^DKV h; k^R = RoPE(W^KR h); output W^O u) --
   "DeepSeek-V3 MLA ... Guide", sections 1-3 of "Core Architecture &
@@ -258,6 +261,27 @@ def attend_absorbed(q_nope, q_rope, rows, w_uk, w_uv, scale, q_pos):
     o = (a.reshape(J * H, L) @ c).reshape(J, H, d_c)               # sum_j a_j c_j
     u = np.einsum("jhc,hdc->jhd", o, w_uv)                         # W^UV_i o_i
     return u, o, m + np.log(l)
+
+
+def merge_partials(o_parts, lse_parts):
+    """Merge attention results taken over disjoint key ranges (split-KV).
+
+    The pages have no split; this is the log-sum-exp identity that makes a
+    split exact in real arithmetic. With lse_s the log of the sum of exp(score)
+    over range s and o_s the softmax-weighted mean of range s's rows, the
+    whole range has lse = log(sum_s exp(lse_s)) and o = sum_s exp(lse_s - lse)
+    o_s. A range without a visible key (lse_s = -inf) gets weight 0.
+    o_parts [S, ..., d], lse_parts [S, ...]; returns (o [..., d], lse [...]).
+    """
+    o_parts = np.asarray(o_parts, np.float64)
+    lse_parts = np.asarray(lse_parts, np.float64)
+    m = lse_parts.max(axis=0)
+    m_ref = np.where(np.isfinite(m), m, 0.0)
+    w = np.exp(lse_parts - m_ref)                      # exp(-inf) = 0
+    tot = w.sum(axis=0)
+    lse = np.where(tot > 0, m_ref + np.log(np.where(tot > 0, tot, 1.0)), -np.inf)
+    o = (w[..., None] * o_parts).sum(axis=0) / np.where(tot > 0, tot, 1.0)[..., None]
+    return o, lse
 
 
 def default_scale(d_nope: int = D_NOPE, d_r: int = D_R) -> float:

@@ -316,6 +316,65 @@ def close_to_printed(x, printed):
     return abs(x - float(printed)) <= 10.0 ** (-digits) + 1e-12
 
 
+def _partial(q_nope, q_rope, rows, w_uk, w_uv, scale, q_pos, a, b):
+    """Attention of every query over keys [a, b) only, through the oracle's
+    unsplit attention on that slice; a query that sees none of them gets
+    o = 0, lse = -inf."""
+    J, H = q_nope.shape[:2]
+    o = np.zeros((J, H, rows.shape[1] - q_rope.shape[-1]))
+    lse = np.full((J, H), -np.inf)
+    for j in range(J):
+        qp = int(q_pos[j]) - a
+        if qp < 0:
+            continue
+        _, oj, lj = O.attend_absorbed(q_nope[j:j + 1], q_rope[j:j + 1], rows[a:b], w_uk, w_uv,
+                                      scale, [qp])
+        o[j], lse[j] = oj[0], lj[0]
+    return o, lse
+
+
+@pytest.mark.parametrize("cuts", [[0, 64, 200], [0, 1, 63, 64, 129, 199, 200], [0, 137, 199, 200]])
+def test_merge_partials_equals_unsplit_attention(cuts):
+    # The split-KV merge (log-sum-exp identity) against the unsplit softmax on
+    # the same keys, including a last range that query 0 cannot see.
+    # Catches: a wrong sign in the weights exp(lse_s - lse), a missing
+    # renormalisation, lse taken as a max instead of a log-sum-exp, an empty
+    # range given weight.
+    rng = np.random.default_rng(11)
+    q_nope, q_rope, rows, w_uk, w_uv, q_pos = rand_case(rng, 2, 3, 200, 512, 64, 128, 128)
+    scale = O.default_scale()
+    _, o_ref, lse_ref = O.attend_absorbed(q_nope, q_rope, rows, w_uk, w_uv, scale, q_pos)
+    parts = [_partial(q_nope, q_rope, rows, w_uk, w_uv, scale, q_pos, a, b)
+             for a, b in zip(cuts[:-1], cuts[1:])]
+    if cuts[-2] == 199:
+        assert np.isneginf(parts[-1][1][0]).all()      # query 0 sees no key of [199, 200)
+    o, lse = O.merge_partials([p[0] for p in parts], [p[1] for p in parts])
+    assert np.max(np.abs(o - o_ref)) <= 1e-12 * np.max(np.abs(o_ref))
+    assert np.max(np.abs(lse - lse_ref)) <= 1e-12 * np.max(np.abs(lse_ref))
+    # the order of the parts does not matter
+    rev = O.merge_partials([p[0] for p in parts[::-1]], [p[1] for p in parts[::-1]])
+    assert np.max(np.abs(rev[0] - o)) <= 1e-13 * np.max(np.abs(o))
+
+
+def test_merge_partials_edge_cases():
+    rng = np.random.default_rng(12)
+    o1 = rng.standard_normal((3, 4, 8))
+    l1 = rng.standard_normal((3, 4))
+    # one part: the identity, exactly
+    o, lse = O.merge_partials([o1], [l1])
+    assert np.array_equal(o, o1) and np.array_equal(lse, l1)
+    # an empty part (lse = -inf, any o) changes nothing
+    o, lse = O.merge_partials([o1, np.full_like(o1, 7.0)], [l1, np.full_like(l1, -np.inf)])
+    assert np.allclose(o, o1, rtol=0, atol=1e-15) and np.allclose(lse, l1, rtol=0, atol=1e-15)
+    # two equal halves of the same keys: same o, lse + log 2
+    o, lse = O.merge_partials([o1, o1], [l1, l1])
+    assert np.allclose(o, o1, rtol=1e-15, atol=1e-15)
+    assert np.allclose(lse, l1 + math.log(2.0), rtol=0, atol=1e-14)
+    # no visible key anywhere: o = 0, lse = -inf
+    o, lse = O.merge_partials([o1, o1], [np.full_like(l1, -np.inf)] * 2)
+    assert not o.any() and np.isneginf(lse).all()
+
+
 def test_cache_footprint_closed_forms():
     g = read_golden("cache_footprint.txt")
     n_h, d_h = 128, 128
