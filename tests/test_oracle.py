@@ -250,7 +250,6 @@ def test_special_cases_closed_form():
     u, o, lse = O.attend_absorbed(q_nope, q_rope, rows_eq, w_uk, w_uv, scale, np.array([6]))
     assert np.allclose(o[0], np.broadcast_to(rows[0, :512], (H, 512)), rtol=1e-13)
     # zero query: uniform weights, o = mean of the visible latents, lse = log L
-    z1, z2 = np.zeros_like(q_nope), np.zeros_like(q_rope)
     for J in (1, 2):
         zq1 = np.zeros((J, H, 128)); zq2 = np.zeros((J, H, 64))
         qp = np.arange(7 - J, 7)
@@ -259,7 +258,6 @@ def test_special_cases_closed_form():
             n = qp[j] + 1
             assert np.allclose(o[j], rows[:n, :512].mean(0), rtol=1e-13)
             assert np.allclose(lse[j], math.log(n), rtol=1e-13)
-    del z1, z2
 
 
 @pytest.mark.parametrize("J", [1, 2])
