@@ -139,12 +139,6 @@ class DecodeSession:
         host_out = torch.empty(self.u.shape, dtype=self.u.dtype).pin_memory()
         return ins, host_in, host_out
 
-    def step_e2e(self, ins, host_in, host_out, stream=None):
-        for d, h in zip(ins, host_in):
-            d.copy_(h, non_blocking=True)
-        self.step(stream)
-        host_out.copy_(self.u, non_blocking=True)
-
     @staticmethod
     def step_io_bytes(ins, host_out) -> tuple:
         return (sum(t.numel() * t.element_size() for t in ins),
