@@ -51,6 +51,7 @@ typedef void *mla_stream_t;    /* cudaStream_t */
 #define MLA_D_V 128    /* per-head value width */
 #define MLA_ROW 576    /* cached elements per token: [c^KV | k^R] */
 #define MLA_PAGE 64    /* tokens per cache page */
+#define MLA_MAX_Q_LEN 16 /* query tokens per sequence in one decode call (MTP verify) */
 
 typedef enum mla_status {
   MLA_OK = 0,
@@ -142,8 +143,9 @@ mla_status_t mla_absorb_q(const mla_bf16_t *q_nope, int ld_qn,
  * the host from the sequence lengths (split-KV: long sequences are cut into
  * several items whose partial results are merged by a log-sum-exp combine).
  * The plan is a flat byte buffer; its size depends only on (batch, q_len,
- * num_ctas) and is returned by mla_plan_bytes. The caller copies the host plan
- * to device memory (cudaMemcpyAsync) and passes both to mla_decode_attention.
+ * num_ctas) and is returned by mla_plan_bytes. mla_plan_upload copies the
+ * host plan to a caller-owned device buffer; mla_decode_attention takes both
+ * copies (the host one for the launch shape, the device one for the kernels).
  */
 typedef struct mla_plan_info {
   int num_items;        /* work items in the plan */
@@ -161,6 +163,11 @@ size_t mla_plan_bytes(int batch, int q_len, int num_ctas);
  * mla_decode_plan -- host.
  *   seq_lens: host int32 [batch], total tokens of each sequence including the
  *             q_len new ones (1 <= q_len <= seq_lens[b]).
+ *   q_len:    query tokens per sequence, 1..MLA_MAX_Q_LEN; query j of
+ *             sequence b sits at position seq_lens[b] - q_len + j and sees the
+ *             keys at positions <= its own (the causal mask between the tokens
+ *             of a multi-token-prediction verify step, "DeepSeek-V3 & MLA in
+ *             2026 ...", section 5).
  *   num_ctas: work lists to balance over; 0 = derive from the current
  *             device's SM count.
  *   max_split: 1 = every (sequence, query) is one item (no combine pass);
@@ -170,11 +177,32 @@ size_t mla_plan_bytes(int batch, int q_len, int num_ctas);
  *             estimated time.
  *   plan:     host buffer of plan_bytes (>= mla_plan_bytes(batch, q_len, num_ctas)).
  *   info:     out, may be NULL.
- * Errors: INVALID_ARGUMENT (bad lengths), WORKSPACE_TOO_SMALL (plan buffer).
+ * Errors: INVALID_ARGUMENT (bad lengths, q_len < 1), UNSUPPORTED (q_len >
+ * MLA_MAX_Q_LEN or n_h outside 16..128 step 16), WORKSPACE_TOO_SMALL (plan
+ * buffer).
  */
 mla_status_t mla_decode_plan(const int32_t *seq_lens, int batch, int q_len, int n_h,
                              int num_ctas, int max_split, void *plan, size_t plan_bytes,
                              mla_plan_info_t *info);
+
+/*
+ * mla_plan_used_bytes -- host. Bytes of a built plan that the kernels read
+ * (header, work lists, items, combine items); 0 if plan_host is NULL or not
+ * a plan.
+ */
+size_t mla_plan_used_bytes(const void *plan_host);
+
+/*
+ * mla_plan_upload -- device copy. Copies the used bytes of the host plan to
+ * plan_dev (cudaMemcpyAsync on `stream`). The host plan must stay unchanged
+ * until the copy has completed (it is read asynchronously when it lives in
+ * page-locked memory).
+ *   plan_dev: device, 16-byte aligned, >= mla_plan_used_bytes(plan_host).
+ * Errors: INVALID_ARGUMENT (NULL, misaligned, not a plan),
+ * WORKSPACE_TOO_SMALL (plan_dev_bytes too small), CUDA.
+ */
+mla_status_t mla_plan_upload(const void *plan_host, void *plan_dev, size_t plan_dev_bytes,
+                             mla_stream_t stream);
 
 /*
  * mla_decode_attention -- device. Absorbed attention over the paged cache:
@@ -196,7 +224,8 @@ mla_status_t mla_decode_plan(const int32_t *seq_lens, int batch, int q_len, int 
  *   lse:         device float32 [batch][q_len][n_h] or NULL.
  * Cache slots past a sequence's length (inside its last page) must hold
  * finite values: they are read, and given weight zero.
- * Supported: n_h % 16 == 0, 16 <= n_h <= 128, 1 <= q_len <= 2.
+ * Supported: n_h % 16 == 0, 16 <= n_h <= 128, 1 <= q_len <= MLA_MAX_Q_LEN (as
+ * the plan).
  */
 mla_status_t mla_decode_attention(const mla_bf16_t *q_full, const mla_bf16_t *cache,
                                   int num_pages, const int32_t *block_table, int max_pages,
@@ -208,16 +237,18 @@ mla_status_t mla_decode_attention(const mla_bf16_t *q_full, const mla_bf16_t *ca
 
 /*
  * mla_decode_attention_noalloc -- device. The same attention as
- * mla_decode_attention, for callers that cannot allocate device memory at the
- * time of the call: code being captured into a CUDA graph, a serving engine
- * that has reserved the GPU's memory for its own cache pool, a plugin running
- * under another framework's allocator. The pages describe no such variant;
- * it exists only for those callers.
+ * mla_decode_attention, for callers that cannot supply device memory of their
+ * own at the time of the call: a serving engine that has reserved the GPU's
+ * memory for its own cache pool, or a plugin running under another
+ * framework's allocator. The pages describe no such variant; it exists only
+ * for those callers.
  * Instead of a caller-supplied workspace, the split-KV partial results go to a
  * fixed 48 MiB array inside the library (allocated on every GPU that loads the
  * library, held until the process exits). The caller still passes all inputs
  * and outputs. The first call on each device looks up the array's address
  * (with that device current); make that first call before any stream capture.
+ * The address is kept per device index for the life of the process: after a
+ * cudaDeviceReset of that device it is stale.
  * Every call shares the array and it keeps the previous call's contents;
  * nothing in it needs to start at zero. Calls that can overlap on the GPU
  * (other streams or host threads) race on the array: serialise them.
@@ -281,6 +312,15 @@ mla_status_t mla_gemm_bf16_ws(const mla_bf16_t *X, int ld_x, const mla_bf16_t *W
  */
 mla_status_t mla_read_status(uint32_t *status, uint32_t *bits, int clear,
                              mla_stream_t stream);
+
+/* mla_check_status -- host. mla_read_status without clearing the word. */
+mla_status_t mla_check_status(uint32_t *status, uint32_t *bits, mla_stream_t stream);
+
+/*
+ * mla_reset_status -- device. Zeroes the status word on `stream`
+ * (cudaMemsetAsync); does not synchronise.
+ */
+mla_status_t mla_reset_status(uint32_t *status, mla_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -87,7 +87,7 @@ extern "C" {
 
 const char *mla_last_error(void) { return g_err; }
 
-int mla_version(void) { return 1; }
+int mla_version(void) { return 2; }
 
 mla_status_t mla_rope_table(float *table, int max_pos, double base) {
   clear_error();
@@ -164,7 +164,9 @@ mla_status_t mla_decode_plan(const int32_t *seq_lens, int batch, int q_len, int 
                              mla_plan_info_t *info) {
   clear_error();
   MLA_CHECK_ARG(batch >= 0, "batch < 0");
-  MLA_CHECK_ARG(q_len >= 1 && q_len <= 2, "q_len must be 1 or 2 (got %d)", q_len);
+  MLA_CHECK_ARG(q_len >= 1, "q_len must be positive (got %d)", q_len);
+  if (q_len > MLA_MAX_Q_LEN)
+    return fail(MLA_ERR_UNSUPPORTED, "q_len = %d (supported: 1..%d)", q_len, MLA_MAX_Q_LEN);
   if (!heads_supported(n_h))
     return fail(MLA_ERR_UNSUPPORTED, "n_h = %d (supported: 16..128, multiple of 16)", n_h);
   MLA_CHECK_ARG(batch == 0 || seq_lens != nullptr, "seq_lens is NULL");
@@ -471,6 +473,39 @@ mla_status_t mla_gemm_bf16_ws(const mla_bf16_t *X, int ld_x, const mla_bf16_t *W
   return launch_projection(X, ld_x, W, ld_w, C, ld_c, c_fp32, M, N, K,
                            use_ws ? static_cast<float *>(workspace) : nullptr,
                            (cudaStream_t)stream);
+}
+
+size_t mla_plan_used_bytes(const void *plan_host) {
+  if (plan_host == nullptr) return 0;
+  const PlanHeader *ph = static_cast<const PlanHeader *>(plan_host);
+  if (ph->magic != kPlanMagic || ph->version != kPlanVersion) return 0;
+  return (size_t)ph->combine_off + (size_t)ph->num_combine * sizeof(CombineItem);
+}
+
+mla_status_t mla_plan_upload(const void *plan_host, void *plan_dev, size_t plan_dev_bytes,
+                             mla_stream_t stream) {
+  clear_error();
+  MLA_CHECK_ARG(plan_host != nullptr && plan_dev != nullptr, "NULL plan pointer");
+  MLA_CHECK_ARG(aligned16(plan_dev), "plan_dev must be 16-byte aligned");
+  const size_t used = mla_plan_used_bytes(plan_host);
+  MLA_CHECK_ARG(used > 0, "not a decode plan");
+  if (plan_dev_bytes < used)
+    return fail(MLA_ERR_WORKSPACE_TOO_SMALL, "device plan buffer %zu B < %zu B", plan_dev_bytes,
+                used);
+  MLA_CUDA_TRY(cudaMemcpyAsync(plan_dev, plan_host, used, cudaMemcpyHostToDevice,
+                               (cudaStream_t)stream));
+  return MLA_OK;
+}
+
+mla_status_t mla_check_status(uint32_t *status, uint32_t *bits, mla_stream_t stream) {
+  return mla_read_status(status, bits, 0, stream);
+}
+
+mla_status_t mla_reset_status(uint32_t *status, mla_stream_t stream) {
+  clear_error();
+  MLA_CHECK_ARG(status != nullptr, "NULL status pointer");
+  MLA_CUDA_TRY(cudaMemsetAsync(status, 0, sizeof(uint32_t), (cudaStream_t)stream));
+  return MLA_OK;
 }
 
 mla_status_t mla_read_status(uint32_t *status, uint32_t *bits, int clear, mla_stream_t stream) {

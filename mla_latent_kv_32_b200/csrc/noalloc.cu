@@ -1,18 +1,20 @@
 // mla_decode_attention_noalloc: the decode attention call for callers that
 // cannot hand the library a workspace.
 //
-// Some callers cannot allocate device memory when they call us: code being
-// recorded into a CUDA graph (cudaMalloc is not a stream operation and breaks
-// the capture), serving engines that reserve nearly all GPU memory up front
-// for their own cache pool and hand out nothing else, and plugins running
-// inside another framework's runtime whose allocator they do not own. For them
-// the split-KV partial results live in one fixed array in this library's own
-// device memory instead of in a caller-supplied workspace.
+// Some callers cannot allocate device memory of their own when they call us:
+// serving engines that reserve nearly all GPU memory up front for their own
+// cache pool and hand out nothing else, and plugins running inside another
+// framework's runtime, whose allocator they do not own and whose memory
+// accounting an extra cudaMalloc would bypass. For them the split-KV partial
+// results live in one fixed array in this library's own device memory instead
+// of in a caller-supplied workspace.
 //
 // The array (kNoAllocScratchBytes, 48 MiB) exists on every GPU that loads the
 // library and stays allocated until the process exits. Its device address is
 // looked up once per device, on the first call made on that device, with that
-// device current; make that first call before any stream capture begins.
+// device current; make that first call before any stream capture begins. The
+// address is kept per device index for the life of the process, so it goes
+// stale if that device is reset (cudaDeviceReset) and the library used again.
 //
 // All calls share the array and it keeps whatever the previous call left in
 // it. Nothing in it has to start at zero: every partial-result slot a call

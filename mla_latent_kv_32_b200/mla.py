@@ -29,6 +29,7 @@ MLA_DEV_TIMEOUT = 0x4
 MLA_DEV_BAD_PLAN = 0x8
 
 D_C, D_R, D_NOPE, D_V, ROW, PAGE = 512, 64, 128, 128, 576, 64
+MAX_Q_LEN = 16
 
 _STATUS_NAMES = {0: "MLA_OK", 1: "MLA_ERR_INVALID_ARGUMENT", 2: "MLA_ERR_UNSUPPORTED",
                  3: "MLA_ERR_WORKSPACE_TOO_SMALL", 4: "MLA_ERR_CUDA", 5: "MLA_ERR_DEVICE"}
@@ -72,6 +73,10 @@ SIGNATURES = {
     "mla_gemm_bf16_workspace_bytes": (_SZ, [_I, _I, _I]),
     "mla_gemm_bf16_ws": (_I, [_P, _I, _P, _I, _P, _I, _I, _I, _I, _I, _P, _SZ, _P]),
     "mla_read_status": (_I, [_P, _P, _I, _P]),
+    "mla_check_status": (_I, [_P, _P, _P]),
+    "mla_reset_status": (_I, [_P, _P]),
+    "mla_plan_used_bytes": (_SZ, [_P]),
+    "mla_plan_upload": (_I, [_P, _P, _SZ, _P]),
 }
 
 _lib: Optional[ctypes.CDLL] = None
@@ -226,3 +231,25 @@ def mla_read_status(status, clear: bool = True, stream=None) -> int:
     if st not in (MLA_OK, MLA_ERR_DEVICE):
         _check(st, "mla_read_status")
     return int(bits.value)
+
+
+def mla_check_status(status, stream=None) -> int:
+    """Returns the device status bits without clearing them."""
+    bits = ctypes.c_uint32(0)
+    st = load().mla_check_status(_ptr(status), ctypes.addressof(bits), _stream(stream))
+    if st not in (MLA_OK, MLA_ERR_DEVICE):
+        _check(st, "mla_check_status")
+    return int(bits.value)
+
+
+def mla_reset_status(status, stream=None):
+    _check(load().mla_reset_status(_ptr(status), _stream(stream)), "mla_reset_status")
+
+
+def mla_plan_used_bytes(plan_host) -> int:
+    return int(load().mla_plan_used_bytes(_ptr(plan_host)))
+
+
+def mla_plan_upload(plan_host, plan_dev, plan_dev_bytes, stream=None):
+    _check(load().mla_plan_upload(_ptr(plan_host), _ptr(plan_dev), int(plan_dev_bytes),
+                                  _stream(stream)), "mla_plan_upload")

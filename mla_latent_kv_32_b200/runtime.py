@@ -71,7 +71,8 @@ class DecodeSession:
         self.rope = to_dev(tab, dev)
         self.plan_host, self.info = mla.mla_decode_plan(inp.lens, self.B, self.q_len, self.n_h,
                                                         num_ctas, max_split)
-        self.plan_dev = to_dev(self.plan_host, dev)
+        self.plan_dev = torch.empty(self.plan_host.nbytes, dtype=torch.uint8, device=dev)
+        mla.mla_plan_upload(self.plan_host, self.plan_dev, self.plan_dev.numel())
         self.ws_bytes = int(self.info.workspace_bytes)
         self.workspace = torch.empty(max(self.ws_bytes, 256), dtype=torch.uint8, device=dev)
         self.q_full = torch.empty((self.T, self.n_h, ROW), dtype=torch.bfloat16, device=dev)
@@ -241,7 +242,8 @@ class LayerSession:
         self.rope = to_dev(mla.mla_rope_table(self.max_pos), dev)
         self.plan_host, self.info = mla.mla_decode_plan(inp.lens, self.B, self.q_len, self.n_h,
                                                         num_ctas, max_split)
-        self.plan_dev = to_dev(self.plan_host, dev)
+        self.plan_dev = torch.empty(self.plan_host.nbytes, dtype=torch.uint8, device=dev)
+        mla.mla_plan_upload(self.plan_host, self.plan_dev, self.plan_dev.numel())
         self.ws_bytes = int(self.info.workspace_bytes)
         self.workspace = torch.empty(max(self.ws_bytes, 256), dtype=torch.uint8, device=dev)
         nq = self.n_h * (D_NOPE + D_R)

@@ -174,7 +174,7 @@ def test_planner_rejects_bad_input():
     with pytest.raises(mla.MlaError):
         mla.mla_decode_plan(np.array([1, 0], np.int32), 2, 1, 128, 8)    # L < q_len
     with pytest.raises(mla.MlaError):
-        mla.mla_decode_plan(np.array([5], np.int32), 1, 3, 128, 8)       # q_len 3
+        mla.mla_decode_plan(np.array([5, 2], np.int32), 2, 3, 128, 8)    # L < q_len 3
     with pytest.raises(mla.MlaError):
         mla.mla_decode_plan(np.array([5], np.int32), 1, 1, 100, 8)       # n_h 100
     buf, info = mla.mla_decode_plan(np.zeros(0, np.int32), 0, 1, 128, 8)
@@ -188,3 +188,33 @@ def test_debug_wait_cap_validated():
     with pytest.raises(mla.MlaError):
         mla.mla_debug_decode_wait(11.0, 0)
     mla.mla_debug_decode_wait(1.0, 0)
+
+
+def test_q_len_range(lib):
+    # MTP verify depths 1..MLA_MAX_Q_LEN are planned; beyond is unsupported,
+    # below one is an invalid argument
+    lens = np.array([40, 300], np.int32)
+    for q_len in (1, 3, 8, mla.MAX_Q_LEN):
+        check_plan(lens, q_len, 7)
+    with pytest.raises(mla.MlaError) as e:
+        mla.mla_decode_plan(np.array([100], np.int32), 1, mla.MAX_Q_LEN + 1, 128, num_ctas=4)
+    assert e.value.status == mla.MLA_ERR_UNSUPPORTED
+    with pytest.raises(mla.MlaError) as e:
+        mla.mla_decode_plan(np.array([100], np.int32), 1, 0, 128, num_ctas=4)
+    assert e.value.status == mla.MLA_ERR_INVALID_ARGUMENT
+
+
+def test_plan_used_bytes_and_upload_checks(lib):
+    lens = np.array([3000, 2000, 77], np.int32)
+    plan, info = mla.mla_decode_plan(lens, 3, 2, 128, num_ctas=5, max_split=0)
+    assert mla.mla_plan_used_bytes(plan) == info.plan_bytes <= plan.nbytes
+    assert mla.mla_plan_used_bytes(np.zeros(64, np.uint8)) == 0
+    with pytest.raises(mla.MlaError) as e:                       # device buffer too small
+        mla.mla_plan_upload(plan, 256, info.plan_bytes - 16, stream=0)
+    assert e.value.status == mla.MLA_ERR_WORKSPACE_TOO_SMALL
+    with pytest.raises(mla.MlaError) as e:                       # misaligned device buffer
+        mla.mla_plan_upload(plan, 258, info.plan_bytes, stream=0)
+    assert e.value.status == mla.MLA_ERR_INVALID_ARGUMENT
+    with pytest.raises(mla.MlaError) as e:
+        mla.mla_reset_status(None, stream=0)
+    assert e.value.status == mla.MLA_ERR_INVALID_ARGUMENT

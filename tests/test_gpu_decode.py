@@ -98,6 +98,11 @@ SMALL = [
     ("heads80_mtp", [130, 2, 513], 2, 80),
     ("heads96", [65, 4100], 1, 96),
     ("heads112_mtp", [257, 66], 2, 112),
+    # multi-token-prediction verify depths beyond two (causal between them)
+    ("mtp3", [3, 64, 66, 700], 3, 128),
+    ("mtp4_heads32", [4, 130, 5000], 4, 32),
+    ("mtp8", [8, 71, 640, 1000], 8, 128),
+    ("mtp16", [16, 64, 300], 16, 64),
 ]
 
 
@@ -111,6 +116,22 @@ def test_decode_small(dev, name, lens, q_len, n_h):
     torch.cuda.synchronize()
     assert sess.read_status() == 0
     check_session(sess, inp, list(range(w.B)), table, nonabs=w.B, check_pool=True)
+
+
+def test_append_bit_exact_with_library_rope_table(dev):
+    # The product path's own RoPE table (mla_rope_table, not the oracle's):
+    # with that same table handed to the oracle, every appended row and every
+    # other slot of the pool is bit-exact.
+    lens = [1, 63, 64, 65, 4000, 300]
+    w = synth.Workload("libtab", B=len(lens), q_len=2, L=max(lens), n_h=128, seed=17)
+    inp = synth.make_decode_inputs(w, lens=[max(l, 2) for l in lens])
+    sess = DecodeSession(inp, dev)                       # rope_table=None: the library's
+    lib_table = mla.mla_rope_table(sess.max_pos)
+    assert np.array_equal(sess.rope.cpu().numpy(), lib_table)
+    sess.step()
+    torch.cuda.synchronize()
+    assert sess.read_status() == 0
+    check_session(sess, inp, list(range(w.B)), lib_table, nonabs=1, check_pool=True)
 
 
 @pytest.mark.parametrize("num_ctas,max_split", [(1, 0), (5, 0), (74, 0), (148, 0), (74, 1)])

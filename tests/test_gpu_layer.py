@@ -50,6 +50,17 @@ def test_layer(dev, name):
     got = np.stack([pool[inp.table[inp.tok_seq[t], inp.tok_pos[t] // 64], inp.tok_pos[t] % 64]
                     for t in ref["new_tok"]])
     assert_parity(O.bf16_to_f64(got), O.bf16_to_f64(ref["new_rows"]), "appended rows")
+    # ... and bit for bit: the GPU's own bf16 projections [c^KV | k^R_pre]
+    # (a GEMM's bf16 output cannot be pinned to float64) through the oracle's
+    # cache row (latent copied, float32 RoPE with the same table) must give
+    # exactly the stored rows, for every token the layer appended
+    kv = bf16_to_numpy_bits(sess.kv)
+    table = mla.mla_rope_table(sess.max_pos)
+    all_tok = np.arange(sess.T)
+    want = O.make_cache_row(kv[:, :512], kv[:, 512:], inp.tok_pos[all_tok], table)
+    got_all = np.stack([pool[inp.table[inp.tok_seq[t], inp.tok_pos[t] // 64],
+                             inp.tok_pos[t] % 64] for t in all_tok])
+    assert np.array_equal(got_all, want), "appended cache rows are not bit-exact"
 
 
 @pytest.mark.parametrize("M,N,K", [(256, 576, 7168), (256, 1536, 7168), (7, 64, 512)])

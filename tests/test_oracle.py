@@ -486,3 +486,162 @@ def test_synth_pool_layout():
         assert np.all(rows[lens[b] - 2:] == synth.FILL_BITS)
     # same seed, same bits
     assert np.array_equal(pool, synth.build_pool(w, lens, table))
+
+
+# ------------------------------------------------- decode_sequence (a step) ---
+
+def _torch_rope_code(k_bits, cos32, sin32):
+    """Cached k^R code through torch's float32 element-wise ops (each product
+    and each sum its own IEEE float32 operation) and torch's bf16 cast."""
+    x = torch.from_numpy(np.asarray(k_bits, np.uint16).view(np.int16)).view(torch.bfloat16)
+    x = x.to(torch.float32)
+    c = torch.from_numpy(np.asarray(cos32, np.float32))
+    s = torch.from_numpy(np.asarray(sin32, np.float32))
+    x0, x1 = x[..., 0::2], x[..., 1::2]
+    a0, b0 = torch.mul(x0, c), torch.mul(x1, s)
+    a1, b1 = torch.mul(x1, c), torch.mul(x0, s)
+    y = torch.empty_like(x)
+    y[..., 0::2] = torch.sub(a0, b0)
+    y[..., 1::2] = torch.add(a1, b1)
+    return y.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def test_rope_f32_code_bit_exact_vs_torch_float32():
+    # The cached k^R code is a fixed function of the bf16 input and the fp32
+    # table: pinned bit for bit to torch's float32 ops. Catches a fused
+    # multiply-add, a rotation evaluated in float64, a pair or sign mix-up.
+    rng = np.random.default_rng(41)
+    n = 20000
+    x = synth.f32_to_bf16_bits((rng.standard_normal((n, 64)) * 3).astype(np.float32))
+    pos = rng.integers(0, 131072, size=n)
+    t = O.rope_table(131072)
+    cs = t[pos]
+    got = O.rope_f32_to_bf16(x, cs[..., 0], cs[..., 1])
+    want = _torch_rope_code(x, cs[..., 0], cs[..., 1])
+    assert np.array_equal(got, want)
+    # the pin separates the float32 contract from an exact (float64) rotation
+    # rounded once: some codes differ between the two
+    exact = O.round_to_bf16(O.rope_f64(O.bf16_to_f64(x), pos))
+    assert (exact != want).any()
+
+
+def _brute_rope(x, p, base=10000.0):
+    d = len(x)
+    y = list(x)
+    for j in range(d // 2):
+        th = p / base ** (2 * j / d)
+        y[2 * j] = x[2 * j] * math.cos(th) - x[2 * j + 1] * math.sin(th)
+        y[2 * j + 1] = x[2 * j + 1] * math.cos(th) + x[2 * j] * math.sin(th)
+    return y
+
+
+def _decode_sequence_case(seed=51, n_pref=3, q_len=2, H=1):
+    """Inputs of a small decode step at the real widths (576-wide rows)."""
+    rng = np.random.default_rng(seed)
+
+    def bf(shape, std=1.0):
+        return synth.f32_to_bf16_bits((rng.standard_normal(shape) * std).astype(np.float32))
+
+    L = n_pref + q_len
+    prefix = bf((n_pref, 576))
+    # the new tokens' latents are large so that the keys appended this step
+    # carry most of the softmax weight
+    c_new = bf((q_len, 512), 3.0)
+    k_new = bf((q_len, 64), 3.0)
+    q_nope = bf((q_len, H, 128))
+    q_pe = bf((q_len, H, 64), 3.0)
+    w_uk = bf((H, 128, 512), 1.0 / math.sqrt(512))
+    w_uv = bf((H, 128, 512), 1.0 / math.sqrt(512))
+    return dict(prefix=prefix, c_new=c_new, k_new=k_new, q_nope=q_nope, q_pe=q_pe, w_uk=w_uk,
+                w_uv=w_uv, L=L)
+
+
+def _decode_sequence_brute(cs):
+    """Independent restatement of one decode step: the new rows built with
+    torch float32 ops at positions L-q_len.., appended after the prefix, the
+    query's RoPE rotated exactly at its own position, then the pure-Python
+    non-absorbed attention."""
+    L, q_len = cs["L"], cs["c_new"].shape[0]
+    tab = O.rope_table(L)
+    pos = np.arange(L - q_len, L)
+    new_k = _torch_rope_code(cs["k_new"], tab[pos][..., 0], tab[pos][..., 1])
+    rows_bits = np.concatenate([cs["prefix"], np.concatenate([cs["c_new"], new_k], 1)], 0)
+    rows = O.bf16_to_f64(rows_bits)
+    qn = O.bf16_to_f64(cs["q_nope"])
+    qp = O.bf16_to_f64(cs["q_pe"])
+    H = qn.shape[1]
+    q_rope = [[_brute_rope(qp[j, h].tolist(), int(pos[j])) for h in range(H)]
+              for j in range(q_len)]
+    u = brute_attention(qn.tolist(), q_rope, rows.tolist(), O.bf16_to_f64(cs["w_uk"]).tolist(),
+                        O.bf16_to_f64(cs["w_uv"]).tolist(), O.default_scale(), pos.tolist())
+    return u, rows_bits
+
+
+def _decode_sequence_error(mod, cs, want_u, want_rows):
+    tab = O.rope_table(cs["L"] + 8)
+    r = mod.decode_sequence(cs["prefix"], cs["c_new"], cs["k_new"], cs["q_nope"], cs["q_pe"],
+                            cs["w_uk"], cs["w_uv"], cs["L"], tab, O.default_scale())
+    err = np.max(np.abs(r["u"] - want_u)) / np.max(np.abs(want_u))
+    return err, np.array_equal(r["rows"], want_rows)
+
+
+@pytest.fixture(scope="module")
+def decode_case():
+    cs = _decode_sequence_case()
+    want_u, want_rows = _decode_sequence_brute(cs)
+    return cs, want_u, want_rows
+
+
+def test_decode_sequence_brute_force(decode_case):
+    # One attention-only decode step with two causal queries: append first,
+    # then score ("DeepSeek-V3 MLA ... Guide", Step 3), q^R rotated at the
+    # query's own position L-2 / L-1.
+    cs, want_u, want_rows = decode_case
+    err, rows_ok = _decode_sequence_error(O, cs, want_u, want_rows)
+    assert rows_ok
+    assert err <= 1e-12
+    # the non-absorbed form of the same step agrees too
+    tab = O.rope_table(cs["L"])
+    r = O.decode_sequence(cs["prefix"], cs["c_new"], cs["k_new"], cs["q_nope"], cs["q_pe"],
+                          cs["w_uk"], cs["w_uv"], cs["L"], tab, O.default_scale(),
+                          form="nonabsorbed")
+    assert np.max(np.abs(r["u"] - want_u)) <= 1e-12 * np.max(np.abs(want_u))
+
+
+def _plant_score_before_append(monkeypatch):
+    real = O.attend_absorbed
+
+    def scored_on_prefix(q_nope, q_rope, rows, w_uk, w_uv, scale, q_pos):
+        n = len(q_pos)
+        return real(q_nope, q_rope, rows[:-n], w_uk, w_uv, scale,
+                    np.minimum(np.asarray(q_pos), len(rows) - n - 1))
+    monkeypatch.setattr(O, "attend_absorbed", scored_on_prefix)
+
+
+def _plant_query_rope_at_last_position(monkeypatch):
+    real = O.rope_f64
+
+    def rope_last(x, pos, base=O.ROPE_BASE):
+        p = np.asarray(pos)
+        return real(x, np.full_like(p, p.max()), base)
+    monkeypatch.setattr(O, "rope_f64", rope_last)
+
+
+def _plant_append_one_position_late(monkeypatch):
+    real = O.make_cache_row
+
+    def late(c, k, pos, table):
+        return real(c, k, np.asarray(pos) + 1, table)
+    monkeypatch.setattr(O, "make_cache_row", late)
+
+
+@pytest.mark.parametrize("plant", [_plant_score_before_append,
+                                   _plant_query_rope_at_last_position,
+                                   _plant_append_one_position_late])
+def test_decode_sequence_pin_catches_planted_mistakes(decode_case, monkeypatch, plant):
+    # Each plausible slip in the step's composition, planted in the oracle,
+    # moves u far outside the 1e-12 pin (or changes the appended rows).
+    cs, want_u, want_rows = decode_case
+    plant(monkeypatch)
+    err, rows_ok = _decode_sequence_error(O, cs, want_u, want_rows)
+    assert err > 1e-4 or not rows_ok
