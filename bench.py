@@ -62,13 +62,25 @@ TRAFFIC = {
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--workload", default="v3")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="override the workload's batch (a smaller case of the same "
+                         "workload, e.g. for profiling)")
     ap.add_argument("--num-ctas", type=int, default=0)
     ap.add_argument("--max-split", type=int, default=-1)
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=200,
+                    help="end-to-end steps timed (at least --steps)")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the per-workload lines (ragged, long_mtp, mtp8, layer_v3, tiny)")
+    ap.add_argument("--configs",
+                    default="tiny,ragged,long_mtp,mtp8,prefill,layer_v3,tiny:folded,"
+                            "layer_v3:folded",
+                    help="comma-separated workloads measured besides the headline one "
+                         "(':folded' = the layer with folded weights)")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--ramp-seconds", type=float, default=0.3,
                     help="back-to-back untimed steps before timing, so the clocks leave "
@@ -413,6 +425,152 @@ def run_rows(args):
     return 0
 
 
+def timed_calls(run, flush, stream, K):
+    """K calls of run(), L2 flushed before each outside the events; per-call
+    device milliseconds (CUDA events on ``stream``)."""
+    import torch
+    ev = []
+    for _ in range(K):
+        if flush is not None:
+            flush()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        run()
+        b.record(stream)
+        ev.append((a, b))
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in ev]
+
+
+def attention_work(inp, w):
+    """(cache bytes read once, FLOPs) of one attention call: 1152 B per cached
+    token, 2176 FLOP per (visible cached token, head, query token)."""
+    cache_bytes = int(inp.lens.sum()) * ROW_BYTES
+    vis = sum(int(L) - w.q_len + j + 1 for L in inp.lens for j in range(w.q_len))
+    return cache_bytes, float(vis) * w.n_h * FLOP_PER_TOKEN_HEAD
+
+
+def roofline_of(nbytes, flops, t_ms, peaks):
+    t_mem = nbytes / (peaks["hbm_gbs"] * 1e9)
+    t_tc = flops / (peaks["bf16_tflops"] * 1e12)
+    t = t_ms / 1e3
+    return {"bound": "hbm" if t_mem >= t_tc else "tensor", "roofline_us": max(t_mem, t_tc) * 1e6,
+            "measured_us": t_ms * 1e3, "frac_of_roofline": max(t_mem, t_tc) / t,
+            "gbs": nbytes / t / 1e9, "tflops": flops / t / 1e12,
+            "frac_spec": max(nbytes / (SPEC_PEAKS["hbm_gbs"] * 1e9),
+                             flops / (SPEC_PEAKS["bf16_tflops"] * 1e12)) / t}
+
+
+def measure_decode_config(name, dev, flush, stream, K, peaks, args):
+    """One attention-only workload: the whole step (one graph replay) and the
+    attention call alone, each after an L2 flush; the roofline of the call."""
+    import torch
+    import synth
+    from mla_latent_kv_32_b200.runtime import DecodeSession
+    w = synth.WORKLOADS[name]
+    inp = synth.make_decode_inputs(w)
+    sess = DecodeSession(inp, dev)
+    for _ in range(3):
+        sess.step()
+    torch.cuda.synchronize()
+    assert sess.read_status() == 0, f"{name}: device status during warm-up"
+    sess.capture()
+    sess.replay(stream)
+    step = timed_calls(lambda: sess.replay(stream), flush, stream, K)
+    attn = timed_calls(sess.attend, flush, stream, K)
+    assert sess.read_status() == 0, f"{name}: device status in the timed calls"
+    nbytes, flops = attention_work(inp, w)
+    t_step, t_attn = statistics.median(step), statistics.median(attn)
+    out = {"workload": workload_config(w, inp, None)["workload"],
+           "tokens_per_s": w.B * w.q_len / (t_step / 1e3), "step_ms": t_step,
+           "attention_ms": t_attn, "step_ms_stats": dist_stats(step),
+           "attention_ms_stats": dist_stats(attn), "cache_bytes": nbytes, "flops": flops,
+           "cache_gbs_attention": nbytes / (t_attn / 1e3) / 1e9,
+           "roofline": roofline_of(nbytes, flops, t_attn, peaks),
+           "plan": {"work_lists": int(sess.info.num_ctas), "items": int(sess.info.num_items),
+                    "partials": int(sess.info.num_partials),
+                    "combine": int(sess.info.num_combine)},
+           "launches_per_step": 4 + (1 if sess.info.num_combine else 0)}
+    if w.q_len > 16:
+        # the same attention in the expanded (non-absorbed) form: 2*(128+64)
+        # + 2*128 FLOP per (visible token, head, query) plus expanding K^C and
+        # V (2 * 2 * 512 * 128 per cached token and head); for context only
+        vis = flops / (w.n_h * FLOP_PER_TOKEN_HEAD)
+        out["flops_expanded_form"] = (vis * w.n_h * (2 * 192 + 2 * 128)
+                                      + float(inp.lens.sum()) * w.n_h * 4 * 512 * 128)
+    del sess
+    torch.cuda.empty_cache()
+    return out
+
+
+def measure_layer_config(name, dev, flush, stream, K, peaks, folded=False):
+    """A whole decode layer from hidden states: the step (one graph replay of
+    the seven library calls) and the attention call alone. For the step the
+    roofline counts the cache, every weight and the activations once, and the
+    projection FLOPs besides the attention's; a launch-bound layer (the tiny
+    one) reports microseconds per step only."""
+    import torch
+    import synth
+    from mla_latent_kv_32_b200.runtime import LayerSession
+    w = synth.WORKLOADS[name]
+    inp = synth.make_layer_inputs(w)
+    ls = LayerSession(inp, dev, folded=folded)
+    for _ in range(3):
+        ls.step()
+    torch.cuda.synchronize()
+    assert ls.read_status() == 0, f"{name}: device status during warm-up"
+    ls.capture()
+    ls.replay(stream)
+    big = w.name != "tiny"
+    step = timed_calls(lambda: ls.replay(stream), flush if big else None, stream, K)
+    attn = timed_calls(ls.attend, flush if big else None, stream, K)
+    assert ls.read_status() == 0, f"{name}: device status in the timed calls"
+    t_step, t_attn = statistics.median(step), statistics.median(attn)
+    cache_bytes = int(inp.lens.sum()) * ROW_BYTES
+    attn_flops = float(sum(int(L) for L in inp.lens)) * w.n_h * FLOP_PER_TOKEN_HEAD
+    Tq, T, H, d = ls.Tq, ls.T, w.n_h, w.hidden
+    ql = w.q_lora
+    q_in = ql or d
+    if folded:
+        # weights the folded step reads: W_DQ, W_QR, W~QK, W_DKV|W_KR, W~O
+        wbytes = 2 * ((ql * d if ql else 0) + H * 64 * q_in + H * 512 * q_in + 576 * d
+                      + d * H * 512)
+        proj_flops = ((2.0 * Tq * ql * d if ql else 0.0) + 2.0 * Tq * H * 64 * q_in
+                      + 2.0 * T * 576 * d + 2.0 * Tq * d * H * 512)
+        absorb_flops = 2.0 * Tq * H * 512 * q_in
+    else:
+        wbytes = sum(int(v.size) for v in inp.weights.values()) * 2
+        if ql:
+            proj_flops = (2.0 * Tq * ql * d + 2.0 * Tq * H * 192 * ql + 2.0 * T * 576 * d
+                          + 2.0 * Tq * d * H * 128)
+        else:
+            proj_flops = 2.0 * Tq * H * 192 * d + 2.0 * T * 576 * d + 2.0 * Tq * d * H * 128
+        absorb_flops = 2.0 * 2 * Tq * H * 128 * 512
+    act_bytes = (T * d + Tq * d * 2 + T * 576) * 2
+    out = {"workload": (f"{w.name}: whole MLA decode layer, batch {w.B}, context {w.L}, hidden "
+                        f"{w.hidden}, q_lora {w.q_lora or 'none'}, n_h {w.n_h}"
+                        + (", folded weights W~QK = W^UK^T W^UQ and W~O = W^O W^UV per head"
+                           if folded else "")),
+           "weight_bytes": wbytes,
+           "tokens_per_s": Tq / (t_step / 1e3), "step_ms": t_step, "attention_ms": t_attn,
+           "step_ms_stats": dist_stats(step), "attention_ms_stats": dist_stats(attn),
+           "launches_per_step": (6 if folded else 7) + (1 if ls.info.num_combine else 0)}
+    if big:
+        out["l2"] = "flushed before every timed call"
+        out["roofline_attention"] = roofline_of(cache_bytes, attn_flops, t_attn, peaks)
+        out["roofline_step"] = roofline_of(cache_bytes + wbytes + act_bytes,
+                                           attn_flops + proj_flops + absorb_flops, t_step, peaks)
+        out["step_bytes"] = cache_bytes + wbytes + act_bytes
+        out["step_flops"] = attn_flops + proj_flops + absorb_flops
+    else:
+        out["us_per_step_graph_replay"] = t_step * 1e3
+        out["l2"] = "not flushed: the layer is launch-bound (0.3 MB of cache)"
+        out["roofline"] = None
+    del ls
+    torch.cuda.empty_cache()
+    return out
+
+
 def main():
     args = parse()
     rank = int(os.environ.get("RANK", "0"))
@@ -428,7 +586,8 @@ def main():
     import synth
     from mla_latent_kv_32_b200 import build as build_mod
     from mla_latent_kv_32_b200 import mla
-    from mla_latent_kv_32_b200.runtime import DecodeSession
+    from mla_latent_kv_32_b200.runtime import (DecodeSession, capture_io_step,
+                                               run_e2e_graphs)
 
     assert torch.cuda.is_available(), "bench.py needs a CUDA device"
     torch.cuda.set_device(local)
@@ -444,11 +603,15 @@ def main():
     mla.load()
 
     w = synth.WORKLOADS[args.workload]
+    if args.batch:
+        import dataclasses
+        w = dataclasses.replace(w, B=args.batch)
     assert not w.layer, "bench.py times the attention-only decode workloads"
     inp = synth.make_decode_inputs(w)
     sess = DecodeSession(inp, dev, num_ctas=args.num_ctas, max_split=args.max_split)
     flush = L2Flush(dev)
     stream = torch.cuda.current_stream()
+    peaks, peak_src = load_peaks()
 
     def barrier():
         if world > 1:
@@ -488,58 +651,75 @@ def main():
             sess.attend()
             ea[k][1].record(stream)
         barrier()
+        bits = sess.read_status()
+        assert bits == 0, f"device status 0x{bits:x} in the timed steps"
+        step_ms = [a.elapsed_time(b) for a, b in ev]
+        attn_ms = [a.elapsed_time(b) for a, b in ea]
+        t_step = sum(step_ms) / K
+        t_attn = sum(attn_ms) / K
+        t_step, t_attn = max_over_ranks([t_step, t_attn], dist, dev, world)
+
+        tokens = w.B * w.q_len
+        value = whole_job_rate(world, tokens, t_step)
+        cache_bytes, flops = attention_work(inp, w)
+
+        # e2e: per-step inputs uploaded from pinned host memory and the result
+        # read back to pinned host memory, through the library's calls. Two
+        # independent sessions (each with its own cache, weights and I/O
+        # buffers) each hold one CUDA graph of upload + four calls + download
+        # and alternate steps on two streams, so one batch's copies overlap
+        # the other's compute. Every step touches more than L2 holds, so no
+        # flush runs in this loop.
+        e2e = None
+        if not args.no_e2e:
+            sess2 = DecodeSession(inp, dev, num_ctas=args.num_ctas, max_split=args.max_split)
+            pair = [sess, sess2]
+            ins, host_in, host_out0 = sess.pinned_step_buffers()
+            host_outs = [host_out0, torch.empty_like(host_out0).pin_memory()]
+            h2d, d2h = DecodeSession.step_io_bytes(ins, host_out0)
+            graphs = [capture_io_step(s_, host_in, host_outs[i]) for i, s_ in enumerate(pair)]
+            streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+            run_e2e_graphs(graphs, streams, 8)
+            torch.cuda.synchronize()
+            E = max(args.e2e_steps, K)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            barrier()
+            e0.record(stream)
+            for s_ in streams:
+                s_.wait_stream(stream)
+            host_s = run_e2e_graphs(graphs, streams, E)
+            for s_ in streams:
+                stream.wait_stream(s_)
+            e1.record(stream)
+            barrier()
+            t_e2e = e0.elapsed_time(e1) / E
+            (t_e2e,) = max_over_ranks([t_e2e], dist, dev, world)
+            for s_ in pair:
+                assert s_.read_status() == 0, "device status in the end-to-end loop"
+            e2e = {"value": whole_job_rate(world, tokens, t_e2e), "unit": UNIT,
+                   "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                   "ms_per_step": t_e2e, "steps": E,
+                   "host_enqueue_us_per_step": host_s / E * 1e6,
+                   "method": "two sessions, each one CUDA graph of upload (pinned host -> "
+                             "device) + the four library calls + download (device -> pinned "
+                             "host); steps alternate on two streams so one batch's copies "
+                             "overlap the other's compute; no L2 flush (each step touches "
+                             "> L2)"}
+            del graphs, sess2
+
+        configs = {}
+        if not args.no_configs and world == 1:
+            for key in [c for c in args.configs.split(",") if c and c != args.workload]:
+                name, _, variant = key.partition(":")
+                wc = synth.WORKLOADS[name]
+                if wc.layer:
+                    configs[key] = measure_layer_config(name, dev, flush, stream, max(5, K // 2),
+                                                        peaks, folded=variant == "folded")
+                else:
+                    configs[key] = measure_decode_config(name, dev, flush, stream,
+                                                         max(5, K // 2), peaks, args)
         clocks.mark_end()
-    bits = sess.read_status()
-    assert bits == 0, f"device status 0x{bits:x} in the timed steps"
-    step_ms = [a.elapsed_time(b) for a, b in ev]
-    attn_ms = [a.elapsed_time(b) for a, b in ea]
-    t_step = sum(step_ms) / K
-    t_attn = sum(attn_ms) / K
-    t_step, t_attn = max_over_ranks([t_step, t_attn], dist, dev, world)
 
-    tokens = w.B * w.q_len
-    value = whole_job_rate(world, tokens, t_step)
-    cache_bytes = int(inp.lens.sum()) * ROW_BYTES
-    # FLOPs: 2176 per (visible cached token, head, query)
-    vis = sum(int(L) - w.q_len + j + 1 for L in inp.lens for j in range(w.q_len))
-    flops = float(vis) * w.n_h * FLOP_PER_TOKEN_HEAD
-
-    # e2e: per-step inputs from pinned host memory, result read back to pinned
-    # host memory, through the library's calls. Two independent sessions
-    # (each with its own 302 MB cache, weights and I/O buffers) alternate
-    # steps, so one batch's uploads and downloads overlap the other's compute;
-    # every step touches more than L2 holds, so no flush runs in this loop.
-    e2e = None
-    if not args.no_e2e:
-        from mla_latent_kv_32_b200.runtime import run_e2e_pipelined
-        sess2 = DecodeSession(inp, dev, num_ctas=args.num_ctas, max_split=args.max_split)
-        pair = [sess, sess2]
-        for s_ in pair:
-            s_.capture()   # one graph launch per step: the loop is not bound by host launches
-        ins, host_in, host_out0 = sess.pinned_step_buffers()
-        host_outs = [host_out0, torch.empty_like(host_out0).pin_memory()]
-        h2d, d2h = DecodeSession.step_io_bytes(ins, host_out0)
-        comp = torch.cuda.current_stream()
-        up_s, down_s = torch.cuda.Stream(), torch.cuda.Stream()
-        run_e2e_pipelined(pair, host_in, host_outs, 4, comp, up_s, down_s)
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        barrier()
-        e0.record(comp)
-        run_e2e_pipelined(pair, host_in, host_outs, K, comp, up_s, down_s)
-        e1.record(comp)
-        barrier()
-        t_e2e = e0.elapsed_time(e1) / K
-        (t_e2e,) = max_over_ranks([t_e2e], dist, dev, world)
-        e2e = {"value": whole_job_rate(world, tokens, t_e2e), "unit": UNIT,
-               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-               "ms_per_step": t_e2e,
-               "method": "two sessions alternate steps (each step one CUDA graph of the four "
-                         "library calls); uploads and downloads overlap the other batch's "
-                         "compute; no L2 flush (each step touches > L2)"}
-        del sess2
-
-    peaks, peak_src = load_peaks()
     gbs = cache_bytes / (t_attn / 1e3) / 1e9
     tfs = flops / (t_attn / 1e3) / 1e12
     t_mem = cache_bytes / (peaks["hbm_gbs"] * 1e9)
@@ -580,6 +760,7 @@ def main():
         "e2e": e2e,
         "gpu_launches": launches_timed,
         "clocks": clocks.summary(),
+        "configs": configs or None,
     }
     if rank == 0 and world == 1 and not args.no_cpu:
         tps, desc, _ = oracle_sample(w, inp, budget_s=12.0)

@@ -51,7 +51,7 @@ typedef void *mla_stream_t;    /* cudaStream_t */
 #define MLA_D_V 128    /* per-head value width */
 #define MLA_ROW 576    /* cached elements per token: [c^KV | k^R] */
 #define MLA_PAGE 64    /* tokens per cache page */
-#define MLA_MAX_Q_LEN 16 /* query tokens per sequence in one decode call (MTP verify) */
+#define MLA_MAX_Q_LEN 1024 /* query tokens per sequence in one call (MTP verify, prefill chunk) */
 
 typedef enum mla_status {
   MLA_OK = 0,
@@ -165,9 +165,11 @@ size_t mla_plan_bytes(int batch, int q_len, int num_ctas);
  *             q_len new ones (1 <= q_len <= seq_lens[b]).
  *   q_len:    query tokens per sequence, 1..MLA_MAX_Q_LEN; query j of
  *             sequence b sits at position seq_lens[b] - q_len + j and sees the
- *             keys at positions <= its own (the causal mask between the tokens
- *             of a multi-token-prediction verify step, "DeepSeek-V3 & MLA in
- *             2026 ...", section 5).
+ *             keys at positions <= its own: the causal mask between the tokens
+ *             of a multi-token-prediction verify step ("DeepSeek-V3 & MLA in
+ *             2026 ...", section 5) or of a chunked-prefill chunk (the causal
+ *             forward of "DeepSeek-V3 MLA ... Guide", Step 2, restricted to the
+ *             chunk's queries, computed in the absorbed form).
  *   num_ctas: work lists to balance over; 0 = derive from the current
  *             device's SM count.
  *   max_split: 1 = every (sequence, query) is one item (no combine pass);
@@ -304,6 +306,47 @@ size_t mla_gemm_bf16_workspace_bytes(int M, int N, int K);
 mla_status_t mla_gemm_bf16_ws(const mla_bf16_t *X, int ld_x, const mla_bf16_t *W, int ld_w,
                               void *C, int ld_c, int c_fp32, int M, int N, int K,
                               void *workspace, size_t workspace_bytes, mla_stream_t stream);
+
+/*
+ * Folded weights ("DeepSeek-V3 MLA: Multi-Head Latent Attention Guide", "The
+ * Matrix Absorption Trick", parts 2-3: W^UK folded into the query side and
+ * W^UV pre-multiplied into the output projection; "Deconstructing DeepSeek V4
+ * Pro ...", "Practical Deployment & Systems Engineering Takeaways": the
+ * query/key up-projection product pre-computed once). Computed once per
+ * weight set; fp32 accumulation, one bf16 rounding per folded element.
+ *
+ * mla_fold_qk -- device.
+ *   W~QK[h*512 + c][i] = sum_d w_uq[(h*128 + d)*ld_uq + i] * w_uk[h][d][c]
+ *   w_uq: device bf16 [n_h*128][ld_uq] (W^UQ, or W_Q of a layer without a
+ *         query latent), q_in input features (q_in % 64 == 0).
+ *   w_uk: device bf16 [n_h][128][512].
+ *   w_qk: device bf16 [n_h*512][q_in], written.
+ *   workspace: device, >= mla_fold_qk_workspace_bytes(n_h) (holds W^UK with
+ *              d contiguous), not in use by another call at the same time.
+ * mla_fold_o -- device.
+ *   W~O[f][h*512 + c] = sum_d w_o[f*ld_o + h*128 + d] * w_uv[h][d][c]
+ *   w_o: device bf16 [d_model][ld_o] (W^O, n_h*128 input features).
+ *   w_uv: device bf16 [n_h][128][512].  w_o_folded: device bf16 [d_model][n_h*512].
+ *   The output projection then runs as mla_gemm_bf16 of o_latent viewed as
+ *   [T][n_h*512] against W~O (K = n_h*512), with no mla_out_absorb.
+ * mla_absorb_q_folded -- device. The query absorption from the folded weight:
+ *   q_full[t][h][0:512]   = sum_i W~QK[h*512 + c][i] * x[t*ld_x + i]
+ *   q_full[t][h][512:576] = RoPE(q_pe[t][h][:], pos[t])   (a copy if pos == NULL)
+ *   x: device bf16, the query input (c^Q, or h without a query latent), k_in
+ *      features (k_in % 64 == 0). Other arguments as mla_absorb_q.
+ * Supported: n_h <= 128 (absorb: 16..128, multiple of 16).
+ * Errors: INVALID_ARGUMENT, UNSUPPORTED, WORKSPACE_TOO_SMALL, CUDA.
+ */
+size_t mla_fold_qk_workspace_bytes(int n_h);
+mla_status_t mla_fold_qk(const mla_bf16_t *w_uq, int ld_uq, int q_in, const mla_bf16_t *w_uk,
+                         int n_h, mla_bf16_t *w_qk, void *workspace, size_t workspace_bytes,
+                         mla_stream_t stream);
+mla_status_t mla_fold_o(const mla_bf16_t *w_o, int ld_o, int d_model, const mla_bf16_t *w_uv,
+                        int n_h, mla_bf16_t *w_o_folded, mla_stream_t stream);
+mla_status_t mla_absorb_q_folded(const mla_bf16_t *x, int ld_x, int k_in, const mla_bf16_t *q_pe,
+                                 int ld_qp, const mla_bf16_t *w_qk, const int32_t *pos,
+                                 const float *rope_table, int max_pos, int T, int n_h,
+                                 mla_bf16_t *q_full, uint32_t *status, mla_stream_t stream);
 
 /*
  * mla_read_status -- host. Synchronises `stream`, copies the device status

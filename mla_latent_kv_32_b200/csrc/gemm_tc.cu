@@ -60,6 +60,7 @@ struct GemmTcArgs {
   float *ws;            // bf16 output split over K: fp32 sums at ((z*N + n)*M + m)
   uint32_t *status;
   int tile_z;           // z extent of the GEMM tiles; CTAs beyond it run the side job
+  int b_shared;         // every batch z reads the same B (its tensor map has one z slice)
   // side job (rope_q_pe == nullptr: none)
   const uint16_t *rope_q_pe;
   int rope_ld_qp;
@@ -206,7 +207,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__
       } else {
         tma_load_3d(a_s, &tm_a, kc * 64, m0, z, bar_full + 8 * s);
       }
-      tma_load_3d(b_s, &tm_b, kc * 64, n0, z, bar_full + 8 * s);
+      tma_load_3d(b_s, &tm_b, kc * 64, n0, g.b_shared ? 0 : z, bar_full + 8 * s);
     }
     for (int s = 0; s < stages; ++s)
       if (armed[s]) wait_bar_g(bar_full + 8 * s, (armed[s] - 1) & 1, g.status);
@@ -327,7 +328,9 @@ mla_status_t launch_gemm_tc(const GemmTcDesc &d, cudaStream_t stream) {
   else         // A element (z, m, k) at A + z*sAz + m*sAm + k
     st = make_map3(&tm_a, d.A, d.K, d.M, d.batch, d.sAm, d.sAz, 128);
   if (st != MLA_OK) return st;
-  st = make_map3(&tm_b, d.B, d.K, d.N, d.batch, d.sBn, d.sBz, BN);
+  const bool b_shared = d.sBz == 0;
+  st = make_map3(&tm_b, d.B, d.K, d.N, b_shared ? 1 : d.batch, d.sBn,
+                 b_shared ? (uint64_t)d.sBn * d.N : d.sBz, BN);
   if (st != MLA_OK) return st;
   GemmTcArgs g;
   g.M = d.M;
@@ -371,6 +374,7 @@ mla_status_t launch_gemm_tc(const GemmTcDesc &d, cudaStream_t stream) {
   g.ws = ws_split ? d.split_ws : nullptr;
   g.status = d.status;
   g.tile_z = d.batch * splits;
+  g.b_shared = b_shared ? 1 : 0;
   g.rope_q_pe = d.rope_q_pe;
   g.rope_ld_qp = d.rope_ld_qp;
   g.rope_pos = d.rope_pos;

@@ -29,7 +29,7 @@ MLA_DEV_TIMEOUT = 0x4
 MLA_DEV_BAD_PLAN = 0x8
 
 D_C, D_R, D_NOPE, D_V, ROW, PAGE = 512, 64, 128, 128, 576, 64
-MAX_Q_LEN = 16
+MAX_Q_LEN = 1024
 
 _STATUS_NAMES = {0: "MLA_OK", 1: "MLA_ERR_INVALID_ARGUMENT", 2: "MLA_ERR_UNSUPPORTED",
                  3: "MLA_ERR_WORKSPACE_TOO_SMALL", 4: "MLA_ERR_CUDA", 5: "MLA_ERR_DEVICE"}
@@ -77,6 +77,10 @@ SIGNATURES = {
     "mla_reset_status": (_I, [_P, _P]),
     "mla_plan_used_bytes": (_SZ, [_P]),
     "mla_plan_upload": (_I, [_P, _P, _SZ, _P]),
+    "mla_fold_qk_workspace_bytes": (_SZ, [_I]),
+    "mla_fold_qk": (_I, [_P, _I, _I, _P, _I, _P, _P, _SZ, _P]),
+    "mla_fold_o": (_I, [_P, _I, _I, _P, _I, _P, _P]),
+    "mla_absorb_q_folded": (_I, [_P, _I, _I, _P, _I, _P, _P, _P, _I, _I, _I, _P, _P, _P]),
 }
 
 _lib: Optional[ctypes.CDLL] = None
@@ -253,3 +257,26 @@ def mla_plan_used_bytes(plan_host) -> int:
 def mla_plan_upload(plan_host, plan_dev, plan_dev_bytes, stream=None):
     _check(load().mla_plan_upload(_ptr(plan_host), _ptr(plan_dev), int(plan_dev_bytes),
                                   _stream(stream)), "mla_plan_upload")
+
+
+def mla_fold_qk_workspace_bytes(n_h: int) -> int:
+    return int(load().mla_fold_qk_workspace_bytes(n_h))
+
+
+def mla_fold_qk(w_uq, ld_uq, q_in, w_uk, n_h, w_qk, workspace, workspace_bytes, stream=None):
+    _check(load().mla_fold_qk(_ptr(w_uq), ld_uq, q_in, _ptr(w_uk), n_h, _ptr(w_qk),
+                              _ptr(workspace), int(workspace_bytes), _stream(stream)),
+           "mla_fold_qk")
+
+
+def mla_fold_o(w_o, ld_o, d_model, w_uv, n_h, w_o_folded, stream=None):
+    _check(load().mla_fold_o(_ptr(w_o), ld_o, d_model, _ptr(w_uv), n_h, _ptr(w_o_folded),
+                             _stream(stream)), "mla_fold_o")
+
+
+def mla_absorb_q_folded(x, ld_x, k_in, q_pe, ld_qp, w_qk, pos, rope_table, max_pos, T, n_h,
+                        q_full, status=None, stream=None):
+    _check(load().mla_absorb_q_folded(_ptr(x), ld_x, k_in, _ptr(q_pe), ld_qp, _ptr(w_qk),
+                                      _ptr(pos), _ptr(rope_table), max_pos, T, n_h,
+                                      _ptr(q_full), _ptr(status), _stream(stream)),
+           "mla_absorb_q_folded")

@@ -34,7 +34,28 @@ def to_dev(arr: np.ndarray, device) -> torch.Tensor:
     return torch.from_numpy(np.ascontiguousarray(arr)).to(device)
 
 
-class DecodeSession:
+class _GraphStep:
+    """Capture of a session's ``step`` (fixed buffers and plan) in a CUDA graph;
+    ``replay(stream)`` then runs the step's library calls as one launch."""
+
+    def capture(self):
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            self.step(side)
+        torch.cuda.current_stream().wait_stream(side)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=side):
+            self.step(side)
+        self.graph = g
+        return g
+
+    def replay(self, stream):
+        with torch.cuda.stream(stream):
+            self.graph.replay()
+
+
+class DecodeSession(_GraphStep):
     """One attention-only decode step per call of ``step()``:
 
         mla_cache_append (RoPE on the new keys, paged scatter)
@@ -110,24 +131,6 @@ class DecodeSession:
     def read_status(self) -> int:
         return mla.mla_read_status(self.status, clear=True)
 
-    def capture(self):
-        """Record one step (the four library calls, fixed buffers and plan) in
-        a CUDA graph; ``replay(stream)`` then runs it as a single launch."""
-        side = torch.cuda.Stream()
-        side.wait_stream(torch.cuda.current_stream())
-        with torch.cuda.stream(side):
-            self.step(side)
-        torch.cuda.current_stream().wait_stream(side)
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=side):
-            self.step(side)
-        self.graph = g
-        return g
-
-    def replay(self, stream):
-        with torch.cuda.stream(stream):
-            self.graph.replay()
-
     # e2e: per-step inputs from pinned host memory, result back to host ----
     def io_inputs(self):
         """Device tensors a step reads that come from the host each step."""
@@ -146,57 +149,44 @@ class DecodeSession:
                 host_out.numel() * host_out.element_size())
 
 
-def run_e2e_pipelined(sessions, host_in, host_outs, steps, comp, h2d, d2h):
-    """End-to-end decode steps with host I/O overlapped across independent batches.
+def capture_io_step(sess, host_in, host_out):
+    """Record one end-to-end step of ``sess`` in a CUDA graph: the upload of
+    the step's inputs from pinned host memory (``host_in``, matching
+    ``sess.io_inputs()``), the library calls of the step, and the download of
+    the result ``u`` into pinned ``host_out``. One replay runs all of it."""
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
 
-    Step k runs on sessions[k % len(sessions)] (each owns its cache, weights,
-    plan and device I/O buffers): the upload of step k+1's inputs (pinned
-    ``host_in``, one list of tensors matching each session's ``io_inputs()``)
-    runs on ``h2d`` while step k computes on ``comp``, and the download of
-    step k's result ``u`` into ``host_outs[k % len(sessions)]`` runs on ``d2h``
-    while step k+1 computes. Every step still moves its inputs host->device and
-    its result device->host; ``comp`` waits for the last download at the end.
-    """
-    n = len(sessions)
-    up = [torch.cuda.Event() for _ in range(n)]
-    done = [torch.cuda.Event() for _ in range(n)]
-    down = [torch.cuda.Event() for _ in range(n)]
-    issued_down = [False] * n
+    def body():
+        for d, h in zip(sess.io_inputs(), host_in):
+            d.copy_(h, non_blocking=True)
+        sess.step(side)
+        host_out.copy_(sess.u, non_blocking=True)
 
-    def upload(k):
-        s = k % n
-        with torch.cuda.stream(h2d):
-            if k >= n:
-                h2d.wait_event(done[s])       # the session's previous step read its inputs
-            for d, h in zip(sessions[s].io_inputs(), host_in):
-                d.copy_(h, non_blocking=True)
-            up[s].record(h2d)
+    with torch.cuda.stream(side):
+        body()                                    # warm-up outside the capture
+    torch.cuda.current_stream().wait_stream(side)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        body()
+    return g
 
-    if steps > 0:
-        upload(0)
+
+def run_e2e_graphs(graphs, streams, steps):
+    """Steps 0..steps-1: step k replays graphs[k % n] on streams[k % n]; each
+    graph holds one session's upload, compute and download, so the sessions'
+    copies overlap each other's compute. Returns the host seconds spent
+    enqueueing."""
+    import time
+    n = len(graphs)
+    t0 = time.perf_counter()
     for k in range(steps):
-        s = k % n
-        if k + 1 < steps:
-            upload(k + 1)
-        comp.wait_event(up[s])
-        if issued_down[s]:
-            comp.wait_event(down[s])          # the previous download of this u finished
-        if getattr(sessions[s], "graph", None) is not None:
-            sessions[s].replay(comp)
-        else:
-            sessions[s].step(comp)
-        done[s].record(comp)
-        with torch.cuda.stream(d2h):
-            d2h.wait_event(done[s])
-            host_outs[s].copy_(sessions[s].u, non_blocking=True)
-            down[s].record(d2h)
-        issued_down[s] = True
-    for s in range(n):
-        if issued_down[s]:
-            comp.wait_event(down[s])
+        with torch.cuda.stream(streams[k % n]):
+            graphs[k % n].replay()
+    return time.perf_counter() - t0
 
 
-class LayerSession:
+class LayerSession(_GraphStep):
     """A whole MLA decode layer from hidden states:
 
         [c^Q =] h W_DQ^T ; [q^C | q^R] = (c^Q or h) [W_UQ|W_QR]^T   (mla_gemm_bf16)
@@ -208,9 +198,10 @@ class LayerSession:
     """
 
     def __init__(self, inp, device="cuda", num_ctas: int = 0, max_split: int = -1,
-                 scale: float = DEFAULT_SCALE):
+                 scale: float = DEFAULT_SCALE, folded: bool = False):
         w = inp.w
         self.w = w
+        self.folded = folded
         dev = self.device = torch.device(device)
         self.B, self.q_len, self.n_h = w.B, w.q_len, w.n_h
         self.Tq = w.B * w.q_len
@@ -259,6 +250,25 @@ class LayerSession:
         self.gemm_ws = None
         self._gemm_ws()   # allocated here, not during a step
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        if folded:
+            self._fold(W)
+
+    def _fold(self, W):
+        """Folded weights, computed once by the library: W~QK (query input ->
+        latent query per head) and W~O (latent outputs -> layer output); the
+        step then skips the content query, mla_out_absorb and u."""
+        dev, n_h = self.device, self.n_h
+        self.q_in = self.q_lora or self.hidden
+        w_up = to_dev_bf16(W["w_uq"] if self.q_lora else W["w_q"], dev)
+        self.w_qr = to_dev_bf16(W["w_qr"], dev)
+        self.w_qk_f = torch.empty((n_h * D_C, self.q_in), dtype=torch.bfloat16, device=dev)
+        self.w_o_f = torch.empty((self.hidden, n_h * D_C), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(mla.mla_fold_qk_workspace_bytes(n_h), dtype=torch.uint8, device=dev)
+        mla.mla_fold_qk(w_up, self.q_in, self.q_in, self.w_uk, n_h, self.w_qk_f, ws, ws.numel())
+        mla.mla_fold_o(self.w_o, n_h * D_V, self.hidden, self.w_uv, n_h, self.w_o_f)
+        torch.cuda.synchronize(dev)
+        del w_up, ws
+        self.q_r = torch.empty((self.Tq, n_h * D_R), dtype=torch.bfloat16, device=dev)
 
     # the layer's calls one by one (step runs them in this order) -------------
     def _gemm_ws(self):
@@ -316,7 +326,41 @@ class LayerSession:
         mla.mla_gemm_bf16(self.u, n_h * D_V, self.w_o, n_h * D_V, self.out, d, 1, self.Tq, d,
                           n_h * D_V, stream)
 
+    # the folded step's own calls ---------------------------------------------
+    def project_q_folded(self, stream=None):
+        n_h, d = self.n_h, self.hidden
+        hq = self.h[self.T - self.Tq:]
+        if self.q_lora:
+            ws = self._gemm_ws()
+            mla.mla_gemm_bf16_ws(hq, d, self.w_dq, d, self.cq, self.q_lora, 0, self.Tq,
+                                 self.q_lora, d, ws, ws.numel(), stream)
+            x, ld = self.cq, self.q_lora
+        else:
+            x, ld = hq, d
+        mla.mla_gemm_bf16(x, ld, self.w_qr, ld, self.q_r, n_h * D_R, 0, self.Tq, n_h * D_R, ld,
+                          stream)
+
+    def absorb_folded(self, stream=None):
+        n_h = self.n_h
+        x, ld = (self.cq, self.q_lora) if self.q_lora else (self.h[self.T - self.Tq:], self.hidden)
+        mla.mla_absorb_q_folded(x, ld, self.q_in, self.q_r, n_h * D_R, self.w_qk_f, self.q_pos,
+                                self.rope, self.max_pos, self.Tq, n_h, self.q_full, self.status,
+                                stream)
+
+    def project_out_folded(self, stream=None):
+        n_h, d = self.n_h, self.hidden
+        mla.mla_gemm_bf16(self.o, n_h * D_C, self.w_o_f, n_h * D_C, self.out, d, 1, self.Tq, d,
+                          n_h * D_C, stream)
+
     def step(self, stream=None):
+        if self.folded:
+            self.project_q_folded(stream)
+            self.project_kv(stream)
+            self.append(stream)
+            self.absorb_folded(stream)
+            self.attend(stream)
+            self.project_out_folded(stream)
+            return
         self.project_q(stream)
         self.project_kv(stream)
         self.append(stream)

@@ -28,6 +28,10 @@ What it computes, and where the pages define it:
 * Split-KV merge of partial results (``merge_partials``): the log-sum-exp
   identity; the pages have no split, so this is the plain reading of a
   combine that is exact in real arithmetic.
+* Folded weights (``fold_qk``, ``fold_o``): W~QK_h = (W^UK_h)^T W^UQ_h and
+  W~O = W^O W^UV per head, applied to the query input and to the latent
+  outputs -- "DeepSeek-V3 MLA ... Guide", "The Matrix Absorption Trick",
+  parts 2 and 3; equal to the unfolded layer in real arithmetic.
 * Whole decode layer (query compression c^Q = W^DQ h, q^C = W^UQ c^Q,
   q^R = RoPE(W^QR c^Q); c^KV = W^DKV h; k^R = RoPE(W^KR h); output W^O u) --
   "DeepSeek-V3 MLA ... Guide", sections 1-3 of "Core Architecture &
@@ -238,6 +242,29 @@ def attend_nonabsorbed(q_nope, q_rope, rows, w_uk, w_uv, scale, q_pos,
     return u, att
 
 
+def attend_latent(q_lat, q_rope, rows, scale, q_pos):
+    """Scores on the latent rows and the softmax-weighted latent sum.
+
+    q_lat [J, H, d_c] (the absorbed content query), q_rope [J, H, d_R],
+    rows [L, d_c + d_R]: score_i = (q_lat . c_i + q^R . k^R_i) * scale over the
+    causal prefix, o = sum_i a_i c_i. Returns o [J, H, d_c] and the
+    natural-log sum-exp of the scaled scores lse [J, H].
+    """
+    q_lat = np.asarray(q_lat, np.float64)
+    q_rope = np.asarray(q_rope, np.float64)
+    rows = np.asarray(rows, np.float64)
+    J, H, d_c = q_lat.shape
+    d_r = q_rope.shape[-1]
+    L = rows.shape[0]
+    c, k_r = rows[:, :d_c], rows[:, d_c:]
+    s = (q_lat.reshape(J * H, d_c) @ c.T
+         + q_rope.reshape(J * H, d_r) @ k_r.T).reshape(J, H, L) * scale
+    vis = causal_visible(q_pos, L)[:, None, :]
+    a, m, l = softmax_masked(s, vis)
+    o = (a.reshape(J * H, L) @ c).reshape(J, H, d_c)               # sum_j a_j c_j
+    return o, m + np.log(l)
+
+
 def attend_absorbed(q_nope, q_rope, rows, w_uk, w_uv, scale, q_pos):
     """Absorbed form over the latent rows.
 
@@ -245,22 +272,43 @@ def attend_absorbed(q_nope, q_rope, rows, w_uk, w_uv, scale, q_pos):
     sum-exp of the scaled scores lse [J, H].
     """
     q_nope = np.asarray(q_nope, np.float64)
-    q_rope = np.asarray(q_rope, np.float64)
-    rows = np.asarray(rows, np.float64)
     w_uk = np.asarray(w_uk, np.float64)
     w_uv = np.asarray(w_uv, np.float64)
-    J, H = q_nope.shape[:2]
-    L = rows.shape[0]
-    d_c, d_r = w_uk.shape[-1], q_rope.shape[-1]
-    c, k_r = rows[:, :d_c], rows[:, d_c:]
     q_lat = np.einsum("jhd,hdc->jhc", q_nope, w_uk)                # (W^UK_i)^T q^C_i
-    s = (q_lat.reshape(J * H, d_c) @ c.T
-         + q_rope.reshape(J * H, d_r) @ k_r.T).reshape(J, H, L) * scale
-    vis = causal_visible(q_pos, L)[:, None, :]
-    a, m, l = softmax_masked(s, vis)
-    o = (a.reshape(J * H, L) @ c).reshape(J, H, d_c)               # sum_j a_j c_j
+    o, lse = attend_latent(q_lat, q_rope, rows, scale, q_pos)
     u = np.einsum("jhc,hdc->jhd", o, w_uv)                         # W^UV_i o_i
-    return u, o, m + np.log(l)
+    return u, o, lse
+
+
+def fold_qk(w_up_bits, w_uk_bits, n_h: int) -> np.ndarray:
+    """Query-side fold, float64: W~QK[h*d_c + c][i] = sum_d W_up[h*d_h + d][i]
+    W^UK[h][d][c], so that q~_h = W~QK_h x straight from the query input x
+    (c^Q, or h without a query latent). W_up is W^UQ (or W_Q), [n_h*d_h, q_in]
+    ("DeepSeek-V3 MLA ... Guide", "The Matrix Absorption Trick", part 2;
+    "Deconstructing DeepSeek V4 Pro ...", "Practical Deployment & Systems
+    Engineering Takeaways": the product computed once, offline)."""
+    w_up = bf16_to_f64(w_up_bits)
+    w_uk = bf16_to_f64(w_uk_bits)
+    d_h, d_c = w_uk.shape[1], w_uk.shape[2]
+    q_in = w_up.shape[1]
+    out = np.empty((n_h * d_c, q_in))
+    for h in range(n_h):
+        out[h * d_c:(h + 1) * d_c] = w_uk[h].T @ w_up[h * d_h:(h + 1) * d_h]
+    return out
+
+
+def fold_o(w_o_bits, w_uv_bits, n_h: int) -> np.ndarray:
+    """Output-side fold, float64: W~O[f][h*d_c + c] = sum_d W^O[f][h*d_v + d]
+    W^UV[h][d][c], so that out = W~O [o_1; ...; o_H] straight from the latent
+    attention outputs ("DeepSeek-V3 MLA ... Guide", "The Matrix Absorption
+    Trick", part 3: W^UV pre-multiplied into the output projection)."""
+    w_o = bf16_to_f64(w_o_bits)
+    w_uv = bf16_to_f64(w_uv_bits)
+    d_v, d_c = w_uv.shape[1], w_uv.shape[2]
+    out = np.empty((w_o.shape[0], n_h * d_c))
+    for h in range(n_h):
+        out[:, h * d_c:(h + 1) * d_c] = w_o[:, h * d_v:(h + 1) * d_v] @ w_uv[h]
+    return out
 
 
 def merge_partials(o_parts, lse_parts):
@@ -293,14 +341,17 @@ def default_scale(d_nope: int = D_NOPE, d_r: int = D_R) -> float:
 
 def decode_sequence(prefix_bits, c_new_bits, k_new_bits, q_nope_bits, q_pe_bits,
                     w_uk_bits, w_uv_bits, L: int, table, scale: float,
-                    form: str = "absorbed", heads=None):
+                    form: str = "absorbed", heads=None, queries=None):
     """One attention-only decode step for one sequence of L tokens.
 
     prefix_bits: the first L-q_len cached rows (uint16 [L-q_len, 576]);
     c_new/k_new: the q_len new tokens' latent and pre-RoPE key (appended at
     positions L-q_len..L-1 before attention); q_nope/q_pe: [q_len, H, .] with
-    q_pe pre-RoPE (rotated here exactly, at the query's position).
-    Returns dict with the full row block and the outputs of the chosen form.
+    q_pe pre-RoPE (rotated here exactly, at the query's position). A chunk of
+    prefill is the same step with q_len = the chunk length.
+    ``queries``: indices j of the query tokens to evaluate (default all; every
+    new row is appended either way). Returns dict with the full row block and
+    the outputs of the chosen form for those queries.
     """
     q_len = np.asarray(q_nope_bits).shape[0]
     pos = np.arange(L - q_len, L)
@@ -308,6 +359,10 @@ def decode_sequence(prefix_bits, c_new_bits, k_new_bits, q_nope_bits, q_pe_bits,
     rows_bits = np.concatenate([np.asarray(prefix_bits, np.uint16).reshape(-1, ROW_ELEMS),
                                 new_rows], axis=0)
     rows = bf16_to_f64(rows_bits)
+    sel = np.arange(q_len) if queries is None else np.asarray(queries, dtype=np.int64)
+    q_nope_bits = np.asarray(q_nope_bits)[sel]
+    q_pe_bits = np.asarray(q_pe_bits)[sel]
+    pos = pos[sel]
     q_nope = bf16_to_f64(q_nope_bits)
     q_rope = rope_f64(bf16_to_f64(q_pe_bits), pos[:, None])
     out = {"rows": rows_bits, "new_rows": new_rows}
@@ -338,13 +393,16 @@ def layer_project(h_bits, weights: Dict[str, np.ndarray], n_h: int, tok_pos):
         c_q = h @ W["w_dq"].T                      # c^Q = W^DQ h
         q_c = c_q @ W["w_uq"].T                    # q^C = W^UQ c^Q
         q_r = c_q @ W["w_qr"].T                    # W^QR c^Q (pre-RoPE)
+        x_q = c_q
     else:
         q_c = h @ W["w_q"].T
         q_r = h @ W["w_qr"].T
+        x_q = h
     c_kv = h @ W["w_dkv"].T                        # c^KV = W^DKV h
     k_r = h @ W["w_kr"].T                          # W^KR h (pre-RoPE)
     tok_pos = np.asarray(tok_pos)
     return {
+        "x_q": x_q,
         "q_nope": q_c.reshape(T, n_h, d_nope),
         "q_rope": rope_f64(q_r.reshape(T, n_h, -1), tok_pos[:, None]),
         "c_kv": c_kv,
@@ -353,14 +411,18 @@ def layer_project(h_bits, weights: Dict[str, np.ndarray], n_h: int, tok_pos):
 
 
 def layer_decode(h_bits, weights, n_h: int, q_len: int, tok_seq, tok_pos, query_tok,
-                 prefix_of, lens, scale: float, seqs: Optional[Sequence[int]] = None):
+                 prefix_of, lens, scale: float, seqs: Optional[Sequence[int]] = None,
+                 fold: Optional[Dict[str, np.ndarray]] = None):
     """Whole decode layer in float64.
 
     prefix_of(b, n) -> uint16 [n, 576] returns the synthetic prefix rows of
     sequence b (rows whose tokens do not enter the layer this step). The rows
     computed from h are rounded to bf16 for storage (the cache is a bf16 cache)
-    before attention. Returns dict(out [B*q_len, hidden] for the chosen
-    sequences' queries, u [.., H, 128], o, lse, new_rows).
+    before attention. With ``fold`` = {"w_qk": W~QK, "w_o": W~O} (float64, see
+    fold_qk / fold_o) the latent query is W~QK x and the output W~O o instead
+    of going through q^C, W^UK, W^UV and W^O. Returns dict(out [B*q_len,
+    hidden] for the chosen sequences' queries, u [.., H, 128], o, lse,
+    new_rows).
     """
     tok_seq = np.asarray(tok_seq)
     tok_pos = np.asarray(tok_pos)
@@ -392,9 +454,16 @@ def layer_decode(h_bits, weights, n_h: int, q_len: int, tok_seq, tok_pos, query_
             rows[:n_pref] = prefix_of(b, n_pref)
         qt = query_tok[b * q_len:(b + 1) * q_len]
         ql = np.array([local[int(t)] for t in qt])
-        u, o, lse = attend_absorbed(pr["q_nope"][ql], pr["q_rope"][ql], bf16_to_f64(rows),
-                                    w_uk, w_uv, scale, tok_pos[qt])
-        outs.append(u.reshape(q_len, -1) @ w_o.T)                   # W^O [u_1; ...; u_H]
+        if fold is None:
+            u, o, lse = attend_absorbed(pr["q_nope"][ql], pr["q_rope"][ql], bf16_to_f64(rows),
+                                        w_uk, w_uv, scale, tok_pos[qt])
+            outs.append(u.reshape(q_len, -1) @ w_o.T)               # W^O [u_1; ...; u_H]
+        else:
+            q_lat = (pr["x_q"][ql] @ fold["w_qk"].T).reshape(q_len, n_h, -1)
+            o, lse = attend_latent(q_lat, pr["q_rope"][ql], bf16_to_f64(rows), scale,
+                                   tok_pos[qt])
+            u = np.einsum("jhc,hdc->jhd", o, w_uv)
+            outs.append(o.reshape(q_len, -1) @ fold["w_o"].T)       # W~O [o_1; ...; o_H]
         us.append(u)
         os_.append(o)
         lses.append(lse)

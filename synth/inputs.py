@@ -103,6 +103,11 @@ WORKLOADS: Dict[str, Workload] = {
     # Full decode layer at V3 dims over an 8192-token context.
     "layer_v3": Workload("layer_v3", B=256, q_len=1, L=8192, n_h=128, layer=True,
                          hidden=7168, q_lora=1536),
+    # Multi-token-prediction verify with eight draft tokens per sequence.
+    "mtp8": Workload("mtp8", B=8, q_len=8, L=32768, n_h=128),
+    # Chunked prefill: a 512-token chunk per sequence appended at the end of a
+    # 4096-token context, every chunk token a causal query.
+    "prefill": Workload("prefill", B=4, q_len=512, L=4096, n_h=128),
 }
 
 

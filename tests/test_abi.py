@@ -193,9 +193,8 @@ def test_debug_wait_cap_validated():
 def test_q_len_range(lib):
     # MTP verify depths 1..MLA_MAX_Q_LEN are planned; beyond is unsupported,
     # below one is an invalid argument
-    lens = np.array([40, 300], np.int32)
-    for q_len in (1, 3, 8, mla.MAX_Q_LEN):
-        check_plan(lens, q_len, 7)
+    for q_len in (1, 3, 8, 16, 512, mla.MAX_Q_LEN):
+        check_plan(np.array([max(40, q_len), q_len + 300], np.int32), q_len, 7)
     with pytest.raises(mla.MlaError) as e:
         mla.mla_decode_plan(np.array([100], np.int32), 1, mla.MAX_Q_LEN + 1, 128, num_ctas=4)
     assert e.value.status == mla.MLA_ERR_UNSUPPORTED

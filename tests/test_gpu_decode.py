@@ -103,6 +103,9 @@ SMALL = [
     ("mtp4_heads32", [4, 130, 5000], 4, 32),
     ("mtp8", [8, 71, 640, 1000], 8, 128),
     ("mtp16", [16, 64, 300], 16, 64),
+    # chunked prefill: every token of the chunk is a causal query
+    ("prefill64", [64, 200, 65], 64, 128),
+    ("prefill128_heads32", [128, 1000, 700], 128, 32),
 ]
 
 
@@ -152,34 +155,35 @@ def test_split_invariance(dev, num_ctas, max_split):
     check_session(sess, inp, list(range(w.B)), table, nonabs=1)
 
 
-def test_e2e_pipelined_matches_oracle(dev):
-    # the benchmark's end-to-end loop: two sessions alternate steps, uploads
-    # and downloads overlap the other batch's compute; every step's result
-    # read back to the host must be the oracle's
-    from mla_latent_kv_32_b200.runtime import run_e2e_pipelined
+def test_e2e_graphs_match_oracle(dev):
+    # the benchmark's end-to-end loop: two sessions, each one CUDA graph of
+    # upload + library calls + download, alternate steps on two streams;
+    # every step's result read back to the host must be the oracle's
+    from mla_latent_kv_32_b200.runtime import capture_io_step, run_e2e_graphs
     lens = [700, 64, 1, 129]
     w = synth.Workload("e2e", B=len(lens), q_len=1, L=max(lens), n_h=128, seed=5)
     inp = synth.make_decode_inputs(w, lens=lens)
     table = O.rope_table(max(lens))
     pair = [DecodeSession(inp, dev, rope_table=table) for _ in range(2)]
     ins, host_in, host_out0 = pair[0].pinned_step_buffers()   # the true inputs
-    for s in pair:   # clobber the device inputs: the loop must upload them
+    for s in pair:   # clobber the device inputs: the graphs must upload them
         for t in s.io_inputs():
             t.zero_()
-    pair[1].capture()   # one session eager, one replaying a captured graph
-    for t in pair[1].io_inputs():
-        t.zero_()
     host_outs = [torch.full_like(host_out0, 7.0).pin_memory() for _ in range(2)]
-    comp = torch.cuda.current_stream()
-    run_e2e_pipelined(pair, host_in, host_outs, 5, comp, torch.cuda.Stream(), torch.cuda.Stream())
+    graphs = [capture_io_step(s, host_in, host_outs[i]) for i, s in enumerate(pair)]
+    for s in pair:
+        for t in s.io_inputs():
+            t.zero_()
+    for h in host_outs:
+        h.fill_(7.0)
+    run_e2e_graphs(graphs, [torch.cuda.Stream(), torch.cuda.Stream()], 5)
     torch.cuda.synchronize()
     for s in pair:
         assert s.read_status() == 0
+    ref = np.stack([oracle_seq(inp, b, table)["u"] for b in range(w.B)])
     for h in host_outs:
         u = h.float().numpy().reshape(w.B, 1, 128, 128)
-        got = [u[b] for b in range(w.B)]
-        ref = [oracle_seq(inp, b, table)["u"] for b in range(w.B)]
-        assert_parity(np.stack(got), np.stack(ref), "u (e2e)")
+        assert_parity(u, ref, "u (e2e)")
 
 
 def test_bad_page_sets_status(dev):
@@ -206,7 +210,39 @@ def test_bad_page_sets_status(dev):
     assert np.all(np.isfinite(sess.u.float().cpu().numpy()))
 
 
-@pytest.mark.parametrize("name", ["v3", "ragged", "long_mtp"])
+def test_prefill_full_size_sampled_queries(dev):
+    # The chunked-prefill workload (4 sequences, 512-token chunks ending a
+    # 4096-token context) in the bench's launch configuration; the oracle
+    # evaluates a sample of each sequence's chunk queries (the first and last
+    # among them), and every appended row is checked bit for bit.
+    w = synth.WORKLOADS["prefill"]
+    inp = synth.make_decode_inputs(w)
+    table = O.rope_table(int(inp.lens.max()))
+    sess = DecodeSession(inp, dev, rope_table=table)
+    sess.step()
+    torch.cuda.synchronize()
+    assert sess.read_status() == 0
+    u = sess.u.float().cpu().numpy().reshape(w.B, w.q_len, w.n_h, 128)
+    o = sess.o.float().cpu().numpy().reshape(w.B, w.q_len, w.n_h, 512)
+    pool = bf16_to_numpy_bits(sess.cache)
+    rng = np.random.default_rng(5)
+    got_u, ref_u, got_o, ref_o = [], [], [], []
+    for b in range(w.B):
+        qs = sorted({0, 1, 63, 64, w.q_len - 1, *rng.choice(w.q_len, 6, replace=False).tolist()})
+        L = int(inp.lens[b])
+        prefix = O.gather_rows(inp.pool, inp.table, b, L - w.q_len)
+        r = O.decode_sequence(prefix, inp.c_new[b], inp.k_new[b], inp.q_nope[b], inp.q_pe[b],
+                              inp.w_uk, inp.w_uv, L, table, SCALE, queries=qs)
+        got_u.append(u[b][qs]); ref_u.append(r["u"])
+        got_o.append(o[b][qs]); ref_o.append(r["o"])
+        for j in range(w.q_len):
+            p = L - w.q_len + j
+            assert np.array_equal(pool[inp.table[b, p // 64], p % 64], r["new_rows"][j])
+    assert_parity(np.concatenate(got_u), np.concatenate(ref_u), "u (prefill)")
+    assert_parity(np.concatenate(got_o), np.concatenate(ref_o), "o_latent (prefill)")
+
+
+@pytest.mark.parametrize("name", ["v3", "ragged", "long_mtp", "mtp8"])
 def test_workload_full_size(dev, name):
     w = synth.WORKLOADS[name]
     inp = synth.make_decode_inputs(w)

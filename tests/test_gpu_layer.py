@@ -82,3 +82,36 @@ def test_split_k_gemm_matches_fp32(dev, M, N, K):
     for g_ in (got, got2):
         err = np.abs(g_ - ref)
         assert err.max() <= 2e-2 * np.abs(ref).max() and err.sum() <= 5e-3 * np.abs(ref).sum()
+
+
+@pytest.mark.parametrize("name", ["tiny", "layer_v3"])
+def test_layer_folded(dev, name):
+    # The layer with folded weights (W~QK = W^UK^T W^UQ per head, W~O = W^O W^UV
+    # per head, computed once by the library): the folds match the oracle's
+    # float64 folds to bf16 rounding, and the layer output matches the
+    # oracle's unfolded layer (the definition) within the decode tolerance.
+    w = synth.WORKLOADS[name]
+    inp = synth.make_layer_inputs(w)
+    sess = LayerSession(inp, dev, folded=True)
+    sess.step()
+    torch.cuda.synchronize()
+    assert sess.read_status() == 0
+    W = inp.weights
+    up = W["w_uq"] if w.q_lora else W["w_q"]
+    wqk = bf16_to_numpy_bits(sess.w_qk_f)
+    wof = bf16_to_numpy_bits(sess.w_o_f)
+    for h in synth.sample_heads(w.n_h, 4):
+        ref_qk = O.fold_qk(up[h * 128:(h + 1) * 128], W["w_uk"][h:h + 1], 1)
+        ref_o = O.fold_o(W["w_o"][:, h * 128:(h + 1) * 128], W["w_uv"][h:h + 1], 1)
+        assert_parity(O.bf16_to_f64(wqk[h * 512:(h + 1) * 512]), ref_qk, f"W~QK head {h}",
+                      tol_max=4e-3, tol_mean=3e-3)
+        assert_parity(O.bf16_to_f64(wof[:, h * 512:(h + 1) * 512]), ref_o, f"W~O head {h}",
+                      tol_max=4e-3, tol_mean=3e-3)
+    seqs = [0] if w.B == 1 else synth.sample_sequences(w, inp.lens, 6)
+    ref = O.layer_decode(inp.h, inp.weights, w.n_h, w.q_len, inp.tok_seq, inp.tok_pos,
+                         inp.query_tok, lambda b, n: synth.prefix_rows(w, b, n), inp.lens,
+                         SCALE, seqs)
+    rows = np.concatenate([np.arange(b * w.q_len, (b + 1) * w.q_len) for b in seqs])
+    assert_parity(sess.out.cpu().numpy()[rows], ref["out"], "folded layer output")
+    o = sess.o.float().cpu().numpy()[rows]
+    assert_parity(o, ref["o"], "latent attention output (folded query)")

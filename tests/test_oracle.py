@@ -645,3 +645,104 @@ def test_decode_sequence_pin_catches_planted_mistakes(decode_case, monkeypatch, 
     plant(monkeypatch)
     err, rows_ok = _decode_sequence_error(O, cs, want_u, want_rows)
     assert err > 1e-4 or not rows_ok
+
+
+# ---------------------------------------------------------------- folding ---
+
+def test_fold_brute_force_tiny():
+    # the two folds are plain per-head products: explicit triple loops.
+    # Catches: a transposed W^UK or W^UV, heads mixed up, the wrong slice of
+    # W^O or W^UQ.
+    rng = np.random.default_rng(61)
+    n_h, d_h, d_c, q_in, d_model = 3, 2, 5, 4, 6
+
+    def bf(shape):
+        return synth.f32_to_bf16_bits(rng.standard_normal(shape).astype(np.float32))
+
+    w_up, w_uk = bf((n_h * d_h, q_in)), bf((n_h, d_h, d_c))
+    w_o, w_uv = bf((d_model, n_h * d_h)), bf((n_h, d_h, d_c))
+    U, K = O.bf16_to_f64(w_up), O.bf16_to_f64(w_uk)
+    Wo, V = O.bf16_to_f64(w_o), O.bf16_to_f64(w_uv)
+    fq = O.fold_qk(w_up, w_uk, n_h)
+    fo = O.fold_o(w_o, w_uv, n_h)
+    for h in range(n_h):
+        for c in range(d_c):
+            for i in range(q_in):
+                want = sum(U[h * d_h + d, i] * K[h, d, c] for d in range(d_h))
+                assert abs(fq[h * d_c + c, i] - want) <= 1e-13
+            for f in range(d_model):
+                want = sum(Wo[f, h * d_h + d] * V[h, d, c] for d in range(d_h))
+                assert abs(fo[f, h * d_c + c] - want) <= 1e-13
+
+
+@pytest.mark.parametrize("q_lora", [0, 5])
+def test_folded_layer_equals_unfolded(q_lora):
+    # Associativity: the layer through W~QK and W~O equals the layer through
+    # q^C, W^UK, W^UV and W^O (the absorption identity carried into the
+    # projections). Catches a fold applied to the wrong input (h instead of
+    # c^Q) or the wrong side of the output projection.
+    rng = np.random.default_rng(70 + q_lora)
+    hid, n_h, d_c = 64, 2, 512
+    T, n_pref = 3, 4
+    L = n_pref + T
+
+    def bf(shape, std=1.0):
+        return synth.f32_to_bf16_bits((rng.standard_normal(shape) * std).astype(np.float32))
+
+    W = {}
+    if q_lora:
+        W["w_dq"] = bf((64, hid), 1 / 8); W["w_uq"] = bf((n_h * 128, 64), 1 / 8)
+        W["w_qr"] = bf((n_h * 64, 64), 1 / 8)
+    else:
+        W["w_q"] = bf((n_h * 128, hid), 1 / 8); W["w_qr"] = bf((n_h * 64, hid), 1 / 8)
+    W["w_dkv"] = bf((d_c, hid), 1 / 8); W["w_kr"] = bf((64, hid), 1 / 8)
+    W["w_uk"] = bf((n_h, 128, d_c), 1 / 22.6); W["w_uv"] = bf((n_h, 128, d_c), 1 / 22.6)
+    W["w_o"] = bf((hid, n_h * 128), 1 / 16)
+    h = bf((T, hid))
+    prefix = bf((n_pref, 576))
+    args = (h, W, n_h, 1, np.zeros(T, np.int32), np.arange(n_pref, L, dtype=np.int32),
+            np.array([T - 1]), lambda b, n: prefix[:n], np.array([L]), O.default_scale())
+    ref = O.layer_decode(*args)
+    fold = {"w_qk": O.fold_qk(W["w_uq"] if q_lora else W["w_q"], W["w_uk"], n_h),
+            "w_o": O.fold_o(W["w_o"], W["w_uv"], n_h)}
+    got = O.layer_decode(*args, fold=fold)
+    assert np.max(np.abs(got["out"] - ref["out"])) <= 1e-11 * np.max(np.abs(ref["out"]))
+    assert np.max(np.abs(got["o"] - ref["o"])) <= 1e-11 * np.max(np.abs(ref["o"]))
+
+
+# -------------------------------------------------------- chunked prefill ---
+
+def test_query_subset_matches_full_step():
+    # decode_sequence(queries=...) evaluates only those queries, with every new
+    # row appended: the same values as the full step's rows
+    cs = _decode_sequence_case(seed=81, n_pref=20, q_len=6, H=2)
+    tab = O.rope_table(cs["L"])
+    args = (cs["prefix"], cs["c_new"], cs["k_new"], cs["q_nope"], cs["q_pe"], cs["w_uk"],
+            cs["w_uv"], cs["L"], tab, O.default_scale())
+    full = O.decode_sequence(*args)
+    sub = O.decode_sequence(*args, queries=[5, 0, 3])
+    assert np.array_equal(sub["rows"], full["rows"])
+    assert np.array_equal(sub["u"], full["u"][[5, 0, 3]])
+    assert np.array_equal(sub["lse"], full["lse"][[5, 0, 3]])
+
+
+def test_chunked_prefill_equals_token_by_token_decode():
+    # A chunk of C tokens attended causally in one step gives, for chunk token
+    # j, what a one-token decode step gives after the tokens before it were
+    # appended one by one: the causal mask inside the chunk, restated as
+    # sequential decoding. Catches a chunk token that sees later chunk tokens,
+    # or a query rotated at the wrong position.
+    C, n_pref, H = 5, 9, 2
+    cs = _decode_sequence_case(seed=83, n_pref=n_pref, q_len=C, H=H)
+    L = n_pref + C
+    tab = O.rope_table(L)
+    chunk = O.decode_sequence(cs["prefix"], cs["c_new"], cs["k_new"], cs["q_nope"], cs["q_pe"],
+                              cs["w_uk"], cs["w_uv"], L, tab, O.default_scale())
+    for j in range(C):
+        before = O.make_cache_row(cs["c_new"][:j], cs["k_new"][:j],
+                                  np.arange(n_pref, n_pref + j), tab)
+        prefix = np.concatenate([cs["prefix"], before], axis=0)
+        one = O.decode_sequence(prefix, cs["c_new"][j:j + 1], cs["k_new"][j:j + 1],
+                                cs["q_nope"][j:j + 1], cs["q_pe"][j:j + 1], cs["w_uk"],
+                                cs["w_uv"], n_pref + j + 1, tab, O.default_scale())
+        assert np.max(np.abs(chunk["u"][j] - one["u"][0])) <= 1e-12 * np.max(np.abs(one["u"]))
