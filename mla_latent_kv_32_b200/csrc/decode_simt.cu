@@ -161,28 +161,47 @@ decode_simt_kernel(DecodeArgs a) {
 }
 
 // Log-sum-exp merge of the parts of one (sequence, query): one CTA of 128
-// threads per (combine item, head), 4 latent dims per thread.
+// threads per (combine item, head), 4 latent dims per thread. Parts are read
+// eight at a time (their lse and float4 slices issued before any is used), so
+// a thread keeps eight loads in flight instead of waiting on one per part.
+constexpr int kCombineBatch = 8;
+
 __global__ void __launch_bounds__(128)
 combine_kernel(DecodeArgs a) {
   const PlanHeader *ph = reinterpret_cast<const PlanHeader *>(a.plan_dev);
   const CombineItem ci = reinterpret_cast<const CombineItem *>(a.plan_dev + ph->combine_off)[blockIdx.x];
   const int h = blockIdx.y;
   const int n_h = a.n_h;
+  const float *lse_base = a.ws_lse + (size_t)ci.first_slot * n_h + h;
   float mx = -INFINITY;
-  for (int s = 0; s < ci.n_parts; ++s)
-    mx = fmaxf(mx, a.ws_lse[(size_t)(ci.first_slot + s) * n_h + h]);
+  for (int s0 = 0; s0 < ci.n_parts; s0 += kCombineBatch) {
+#pragma unroll
+    for (int u = 0; u < kCombineBatch; ++u)
+      if (s0 + u < ci.n_parts) mx = fmaxf(mx, __ldg(lse_base + (size_t)(s0 + u) * n_h));
+  }
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   float wsum = 0.f;
-  for (int s = 0; s < ci.n_parts; ++s) {
-    const size_t slot = (size_t)(ci.first_slot + s);
-    const float ls = a.ws_lse[slot * n_h + h];
-    const float w = (ls == -INFINITY) ? 0.f : expf(ls - mx);
-    wsum += w;
-    const float4 v = reinterpret_cast<const float4 *>(a.ws_o + (slot * n_h + h) * MLA_D_C)[threadIdx.x];
-    acc.x = fmaf(w, v.x, acc.x);
-    acc.y = fmaf(w, v.y, acc.y);
-    acc.z = fmaf(w, v.z, acc.z);
-    acc.w = fmaf(w, v.w, acc.w);
+  for (int s0 = 0; s0 < ci.n_parts; s0 += kCombineBatch) {
+    float ls[kCombineBatch];
+    float4 v[kCombineBatch];
+#pragma unroll
+    for (int u = 0; u < kCombineBatch; ++u) {
+      if (s0 + u >= ci.n_parts) continue;
+      const size_t slot = (size_t)(ci.first_slot + s0 + u);
+      ls[u] = __ldg(lse_base + (size_t)(s0 + u) * n_h);
+      v[u] = __ldg(reinterpret_cast<const float4 *>(a.ws_o + (slot * n_h + h) * MLA_D_C) +
+                   threadIdx.x);
+    }
+#pragma unroll
+    for (int u = 0; u < kCombineBatch; ++u) {
+      if (s0 + u >= ci.n_parts) continue;
+      const float w = (ls[u] == -INFINITY) ? 0.f : expf(ls[u] - mx);
+      wsum += w;
+      acc.x = fmaf(w, v[u].x, acc.x);
+      acc.y = fmaf(w, v[u].y, acc.y);
+      acc.z = fmaf(w, v[u].z, acc.z);
+      acc.w = fmaf(w, v[u].w, acc.w);
+    }
   }
   const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
   const size_t row = ((size_t)ci.b * a.q_len + ci.j) * n_h + h;
