@@ -28,6 +28,11 @@ What it computes, and where the pages define it:
 * Split-KV merge of partial results (``merge_partials``): the log-sum-exp
   identity; the pages have no split, so this is the plain reading of a
   combine that is exact in real arithmetic.
+* FP8 latent cache (``quantize_latent_fp8``, ``make_cache_row_fp8``,
+  ``dequant_fp8_rows``, ``decode_sequence_fp8``): E4M3 latent codes with a
+  power-of-two per-token scale, bf16 k^R -- "Deconstructing DeepSeek V4 Pro
+  ...", "Practical Deployment & Systems Engineering Takeaways"; the attention
+  then runs on the exactly dequantized rows.
 * Folded weights (``fold_qk``, ``fold_o``): W~QK_h = (W^UK_h)^T W^UQ_h and
   W~O = W^O W^UV per head, applied to the query input and to the latent
   outputs -- "DeepSeek-V3 MLA ... Guide", "The Matrix Absorption Trick",
@@ -195,6 +200,92 @@ def gather_rows(pool, block_table, b: int, L: int) -> np.ndarray:
     return pages[:L]
 
 
+# ------------------------------------------------------------ FP8 cache ---
+# An 8-bit latent cache ("Deconstructing DeepSeek V4 Pro ...", "Practical
+# Deployment & Systems Engineering Takeaways", quantization strategies: c^KV
+# tolerates E4M3 / E5M2; "DeepSeek-V3 MLA ... Guide", "4. Cache Footprint
+# Math", an FP8 cache). The pages fix no format; the reading taken here: the
+# 512 latent values of a token are E4M3 codes with one power-of-two float32
+# scale per token, the decoupled key k^R stays the bf16 code of the bf16 cache
+# (its rotation carries the position), so a row is 512 + 128 bytes and the
+# scale lives in a separate array.
+
+E4M3_MAX = 448.0
+
+
+def e4m3_round(v) -> np.ndarray:
+    """Round float64 values to the nearest E4M3 value (ties to even),
+    saturating at +-448. E4M3: 1 sign, 4 exponent (bias 7), 3 mantissa bits;
+    normals 2^-6 .. 448, subnormals multiples of 2^-9."""
+    v = np.asarray(v, dtype=np.float64)
+    a = np.abs(v)
+    e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    e = np.maximum(e, -6.0)                       # below 2^-6 the spacing stays 2^-9
+    step = 2.0 ** (e - 3)
+    r = np.rint(a / step) * step                  # rint: ties to even
+    r = np.minimum(r, E4M3_MAX)
+    return np.copysign(r, v)
+
+
+def e4m3_bits(v) -> np.ndarray:
+    """Bit patterns (uint8) of values that are exactly E4M3 (see e4m3_round)."""
+    v = np.asarray(v, dtype=np.float64)
+    a = np.abs(v)
+    sign = (v < 0) | ((v == 0) & np.signbit(v))
+    e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    normal = a >= 2.0 ** -6
+    exp_field = np.where(normal, e + 7, 0).astype(np.int64)
+    mant = np.where(normal, a / 2.0 ** e - 1.0, a / 2.0 ** -6) * 8.0
+    mant = np.rint(mant).astype(np.int64)
+    return ((sign.astype(np.int64) << 7) | (exp_field << 3) | mant).astype(np.uint8)
+
+
+def e4m3_value(bits) -> np.ndarray:
+    """float64 value of E4M3 bit patterns (uint8), the finite codes."""
+    b = np.asarray(bits, dtype=np.uint8).astype(np.int64)
+    s = np.where(b & 0x80, -1.0, 1.0)
+    ef = (b >> 3) & 0xF
+    m = b & 0x7
+    val = np.where(ef == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * 2.0 ** (ef - 7.0))
+    return s * val
+
+
+def fp8_token_scale(amax) -> np.ndarray:
+    """The power of two 2^k with the least k such that amax / 2^k <= 448
+    (1 when amax is 0): the per-token scale of the FP8 cache."""
+    amax = np.asarray(amax, dtype=np.float64)
+    m, e = np.frexp(np.where(amax > 0, amax, 1.0))      # amax = m 2^e, m in [0.5, 1)
+    k = np.where(m <= E4M3_MAX / 512.0, e - 9, e - 8)
+    return np.where(amax > 0, np.ldexp(1.0, k), 1.0)
+
+
+def quantize_latent_fp8(c_kv_bits):
+    """Per token: scale = fp8_token_scale(max |c|), codes = E4M3(c / scale).
+    Returns (codes uint8 [n, 512], scales float64 [n])."""
+    c = bf16_to_f64(np.asarray(c_kv_bits, np.uint16).reshape(-1, D_C))
+    scale = fp8_token_scale(np.abs(c).max(axis=1))
+    codes = e4m3_bits(e4m3_round(c / scale[:, None]))   # division by 2^k is exact
+    return codes, scale
+
+
+def make_cache_row_fp8(c_kv_bits, k_pe_bits, pos, table):
+    """New FP8 cache rows: (bytes uint8 [n, 640] = [512 E4M3 codes | k^R as
+    the bf16 code of make_cache_row, little-endian], scales float64 [n])."""
+    codes, scale = quantize_latent_fp8(c_kv_bits)
+    kr = make_cache_row(c_kv_bits, k_pe_bits, pos, table)[:, D_C:]
+    kr_bytes = np.ascontiguousarray(kr.astype("<u2")).view(np.uint8).reshape(-1, 2 * D_R)
+    return np.concatenate([codes, kr_bytes], axis=1), scale
+
+
+def dequant_fp8_rows(row_bytes, scales) -> np.ndarray:
+    """float64 rows [n, 576] of FP8 cache rows: latent = code * scale (exact),
+    k^R = the stored bf16 values."""
+    row_bytes = np.asarray(row_bytes, np.uint8).reshape(-1, D_C + 2 * D_R)
+    lat = e4m3_value(row_bytes[:, :D_C]) * np.asarray(scales, np.float64).reshape(-1, 1)
+    kr = bf16_to_f64(np.ascontiguousarray(row_bytes[:, D_C:]).view("<u2"))
+    return np.concatenate([lat, kr], axis=1)
+
+
 # -------------------------------------------------------------- attention ---
 
 def softmax_masked(s: np.ndarray, visible: np.ndarray):
@@ -338,6 +429,27 @@ def default_scale(d_nope: int = D_NOPE, d_r: int = D_R) -> float:
 
 
 # ------------------------------------------------------- attention step ----
+
+def decode_sequence_fp8(prefix_bytes, prefix_scales, c_new_bits, k_new_bits, q_nope_bits,
+                        q_pe_bits, w_uk_bits, w_uv_bits, L: int, table, scale: float,
+                        queries=None):
+    """One decode step over an FP8 cache: the new tokens are quantized and
+    appended (make_cache_row_fp8), every row is dequantized exactly, then the
+    absorbed attention of decode_sequence runs on those values."""
+    q_len = np.asarray(q_nope_bits).shape[0]
+    pos = np.arange(L - q_len, L)
+    new_rows, new_scales = make_cache_row_fp8(c_new_bits, k_new_bits, pos, table)
+    rows_b = np.concatenate([np.asarray(prefix_bytes, np.uint8).reshape(-1, D_C + 2 * D_R),
+                             new_rows], axis=0)
+    scales = np.concatenate([np.asarray(prefix_scales, np.float64).reshape(-1), new_scales])
+    rows = dequant_fp8_rows(rows_b, scales)
+    sel = np.arange(q_len) if queries is None else np.asarray(queries, dtype=np.int64)
+    q_nope = bf16_to_f64(np.asarray(q_nope_bits)[sel])
+    q_rope = rope_f64(bf16_to_f64(np.asarray(q_pe_bits)[sel]), pos[sel][:, None])
+    u, o, lse = attend_absorbed(q_nope, q_rope, rows, bf16_to_f64(w_uk_bits),
+                                bf16_to_f64(w_uv_bits), scale, pos[sel])
+    return {"new_rows": new_rows, "new_scales": new_scales, "u": u, "o": o, "lse": lse}
+
 
 def decode_sequence(prefix_bits, c_new_bits, k_new_bits, q_nope_bits, q_pe_bits,
                     w_uk_bits, w_uv_bits, L: int, table, scale: float,

@@ -746,3 +746,74 @@ def test_chunked_prefill_equals_token_by_token_decode():
                                 cs["q_nope"][j:j + 1], cs["q_pe"][j:j + 1], cs["w_uk"],
                                 cs["w_uv"], n_pref + j + 1, tab, O.default_scale())
         assert np.max(np.abs(chunk["u"][j] - one["u"][0])) <= 1e-12 * np.max(np.abs(one["u"]))
+
+
+# -------------------------------------------------------------- FP8 cache ---
+
+def test_e4m3_rounding_matches_torch_float8():
+    # E4M3 rounding (nearest, ties to even, subnormals, signed zero) and the
+    # bit layout, against torch's float8_e4m3fn cast (finite range only: torch
+    # maps values >= 464 to NaN where the cache saturates at 448).
+    rng = np.random.default_rng(90)
+    v = np.concatenate([rng.standard_normal(200000) * 60, rng.standard_normal(20000) * 0.01,
+                        np.array([0.0, -0.0, 448.0, 447.9, 2.0 ** -10, 3 * 2.0 ** -10,
+                                  -(2.0 ** -9), 2.0 ** -6, 1.0625, 1.1875, -2.0 ** -11])])
+    v = v[np.abs(v) < 464]
+    got = O.e4m3_round(v)
+    t = torch.from_numpy(v).to(torch.float8_e4m3fn)
+    assert np.array_equal(got, t.to(torch.float64).numpy())
+    assert np.array_equal(O.e4m3_bits(got), t.view(torch.uint8).numpy())
+    codes = np.array([b for b in range(256) if (b & 0x7F) != 0x7F], np.uint8)   # finite codes
+    want = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(O.e4m3_value(codes), want)
+    assert O.e4m3_round(np.array([460.0, 1e6]))[0] == 448.0      # saturation
+
+
+def test_fp8_scale_and_error_bound():
+    # The per-token scale is the least power of two that brings max|c| to at
+    # most 448 (so max|c|/scale is in (224, 448]); every dequantized value is
+    # within one E4M3 rounding of the bf16 input.
+    rng = np.random.default_rng(91)
+    c = synth.f32_to_bf16_bits((rng.standard_normal((300, 512))
+                                * np.exp(rng.uniform(-12, 12, (300, 1)))).astype(np.float32))
+    codes, scale = O.quantize_latent_fp8(c)
+    x = O.bf16_to_f64(c)
+    amax = np.abs(x).max(1)
+    assert np.all(np.log2(scale) == np.round(np.log2(scale)))
+    r = amax / scale
+    assert np.all(r <= 448.0) and np.all(r > 224.0)
+    deq = O.e4m3_value(codes) * scale[:, None]
+    normal = np.abs(x) / scale[:, None] >= 2.0 ** -6
+    err = np.abs(deq - x)
+    assert np.all(err[normal] <= 2.0 ** -4 * np.abs(x[normal]))
+    assert np.all(err[~normal] <= (2.0 ** -10 * np.broadcast_to(scale[:, None], x.shape))[~normal])
+    zc, zs = O.quantize_latent_fp8(np.zeros((1, 512), np.uint16))
+    assert zs[0] == 1.0 and not zc.any()
+
+
+def test_fp8_decode_equals_bf16_decode_on_representable_rows():
+    # When every latent value is an E4M3 value times a power of two, the FP8
+    # cache is lossless: the FP8 step must equal the bf16 step on the same
+    # inputs (the new rows' k^R code is the bf16 cache's code).
+    rng = np.random.default_rng(92)
+    L, q_len, H = 40, 2, 3
+    lat = O.e4m3_round(rng.standard_normal((L, 512)) * 100) * 2.0 ** -7
+    kr = rng.standard_normal((L, 64))
+    rows_bits = np.concatenate([O.round_to_bf16(lat), O.round_to_bf16(kr)], axis=1)
+    assert np.array_equal(O.bf16_to_f64(rows_bits[:, :512]), lat)
+    prefix = rows_bits[:L - q_len]
+    c_new, k_new = rows_bits[L - q_len:, :512], rows_bits[L - q_len:, 512:]
+    q_nope = O.round_to_bf16(rng.standard_normal((q_len, H, 128)))
+    q_pe = O.round_to_bf16(rng.standard_normal((q_len, H, 64)))
+    w_uk = O.round_to_bf16(rng.standard_normal((H, 128, 512)) / 22.6)
+    w_uv = O.round_to_bf16(rng.standard_normal((H, 128, 512)) / 22.6)
+    tab = O.rope_table(L)
+    ref = O.decode_sequence(prefix, c_new, k_new, q_nope, q_pe, w_uk, w_uv, L, tab,
+                            O.default_scale())
+    pb, ps = O.quantize_latent_fp8(prefix[:, :512])
+    prefix8 = np.concatenate([pb, np.ascontiguousarray(prefix[:, 512:].astype("<u2"))
+                              .view(np.uint8).reshape(-1, 128)], axis=1)
+    got = O.decode_sequence_fp8(prefix8, ps, c_new, k_new, q_nope, q_pe, w_uk, w_uv, L, tab,
+                                O.default_scale())
+    assert np.max(np.abs(got["u"] - ref["u"])) <= 1e-12 * np.max(np.abs(ref["u"]))
+    assert np.array_equal(got["new_rows"][:, 512:].view("<u2"), ref["new_rows"][:, 512:])
