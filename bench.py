@@ -38,6 +38,7 @@ sys.path.insert(0, ROOT)
 METRIC = "MLA decode tokens/sec and cache GB/s (% of HBM/bf16 roofline) on 1 B200"
 UNIT = "tokens/s"
 ROW_BYTES = 1152                 # 576 bf16 per cached token
+FP8_TOKEN_BYTES = 644            # FP8 cache: 512 E4M3 + 64 bf16 + a float32 scale
 FLOP_PER_TOKEN_HEAD = 2 * 576 + 2 * 512
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # B200 data-sheet figures (dense bf16), reported beside the measured peaks
@@ -78,7 +79,7 @@ def parse():
                     help="skip the per-workload lines (ragged, long_mtp, mtp8, layer_v3, tiny)")
     ap.add_argument("--configs",
                     default="tiny,ragged,long_mtp,mtp8,prefill,layer_v3,tiny:folded,"
-                            "layer_v3:folded",
+                            "layer_v3:folded,v3:fp8,ragged:fp8",
                     help="comma-separated workloads measured besides the headline one "
                          "(':folded' = the layer with folded weights)")
     ap.add_argument("--no-cpu", action="store_true")
@@ -461,15 +462,16 @@ def roofline_of(nbytes, flops, t_ms, peaks):
                              flops / (SPEC_PEAKS["bf16_tflops"] * 1e12)) / t}
 
 
-def measure_decode_config(name, dev, flush, stream, K, peaks, args):
+def measure_decode_config(name, dev, flush, stream, K, peaks, args, fp8=False):
     """One attention-only workload: the whole step (one graph replay) and the
-    attention call alone, each after an L2 flush; the roofline of the call."""
+    attention call alone, each after an L2 flush; the roofline of the call.
+    fp8: the same workload over the FP8 cache (644 bytes per cached token)."""
     import torch
     import synth
     from mla_latent_kv_32_b200.runtime import DecodeSession
     w = synth.WORKLOADS[name]
     inp = synth.make_decode_inputs(w)
-    sess = DecodeSession(inp, dev)
+    sess = DecodeSession(inp, dev, fp8=fp8)
     for _ in range(3):
         sess.step()
     torch.cuda.synchronize()
@@ -480,8 +482,11 @@ def measure_decode_config(name, dev, flush, stream, K, peaks, args):
     attn = timed_calls(sess.attend, flush, stream, K)
     assert sess.read_status() == 0, f"{name}: device status in the timed calls"
     nbytes, flops = attention_work(inp, w)
+    if fp8:
+        nbytes = int(inp.lens.sum()) * FP8_TOKEN_BYTES
     t_step, t_attn = statistics.median(step), statistics.median(attn)
-    out = {"workload": workload_config(w, inp, None)["workload"],
+    out = {"workload": workload_config(w, inp, None)["workload"]
+           + (", FP8 (E4M3) latent cache, bf16 k^R, per-token power-of-two scale" if fp8 else ""),
            "tokens_per_s": w.B * w.q_len / (t_step / 1e3), "step_ms": t_step,
            "attention_ms": t_attn, "step_ms_stats": dist_stats(step),
            "attention_ms_stats": dist_stats(attn), "cache_bytes": nbytes, "flops": flops,
@@ -717,7 +722,8 @@ def main():
                                                         peaks, folded=variant == "folded")
                 else:
                     configs[key] = measure_decode_config(name, dev, flush, stream,
-                                                         max(5, K // 2), peaks, args)
+                                                         max(5, K // 2), peaks, args,
+                                                         fp8=variant == "fp8")
         clocks.mark_end()
 
     gbs = cache_bytes / (t_attn / 1e3) / 1e9

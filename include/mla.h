@@ -266,6 +266,44 @@ mla_status_t mla_decode_attention_noalloc(const mla_bf16_t *q_full, const mla_bf
                                           float *lse, uint32_t *status, mla_stream_t stream);
 
 /*
+ * FP8 latent cache ("Deconstructing DeepSeek V4 Pro ...", "Practical
+ * Deployment & Systems Engineering Takeaways": the latent c^KV tolerates
+ * E4M3; "DeepSeek-V3 MLA ... Guide", "4. Cache Footprint Math": an FP8
+ * cache). Layout: cache8 [num_pages][64][640] bytes, a row being
+ *   bytes [0, 512)   the 512 latent values as E4M3 codes, code = E4M3(c / s)
+ *                    (round to nearest even, saturating at 448),
+ *   bytes [512, 640) the rotated k^R as the same 64 bf16 codes the bf16 cache
+ *                    stores (little-endian),
+ * and scales [num_pages][64] float32: s = the least power of two 2^k with
+ * max|c| / 2^k <= 448 (1 when the latent is all zero), so c / s and code * s
+ * are exact. 640 + 4 bytes per token against 1152 for the bf16 cache.
+ *
+ * mla_cache_append_fp8 -- device. mla_cache_append for the FP8 cache: the
+ * row and the scale of each new token are written to its page slot (same
+ * placement, RoPE and error behaviour as mla_cache_append).
+ *   cache: device, 16-byte aligned, updated in place. scales: device float32
+ *   [num_pages][64], 16-byte aligned, updated in place.
+ *
+ * mla_decode_attention_fp8 -- device. mla_decode_attention over the FP8
+ * cache: the same result for the dequantized rows (code * s, k^R); the same
+ * plan, workspace, outputs and errors. Every operand that enters the tensor
+ * cores is the exact dequantized value in bf16.
+ */
+mla_status_t mla_cache_append_fp8(uint8_t *cache, float *scales, int num_pages,
+                                  const int32_t *block_table, int batch, int max_pages,
+                                  const int32_t *seq_idx, const int32_t *pos,
+                                  const mla_bf16_t *c_kv, int ld_c, const mla_bf16_t *k_pe,
+                                  int ld_k, const float *rope_table, int max_pos, int n_tokens,
+                                  uint32_t *status, mla_stream_t stream);
+mla_status_t mla_decode_attention_fp8(const mla_bf16_t *q_full, const uint8_t *cache,
+                                      const float *scales, int num_pages,
+                                      const int32_t *block_table, int max_pages, int batch,
+                                      int q_len, int n_h, float scale, const void *plan_host,
+                                      const void *plan_dev, void *workspace,
+                                      size_t workspace_bytes, mla_bf16_t *o_latent,
+                                      float *lse, uint32_t *status, mla_stream_t stream);
+
+/*
  * mla_out_absorb -- device. Expands the latent attention output through W^UV:
  *   u[t][h*128 + d] = sum_c o_latent[t][h][c] * w_uv[h][d][c]
  * ("DeepSeek-V3 MLA ... Guide", "The Matrix Absorption Trick", part 3:

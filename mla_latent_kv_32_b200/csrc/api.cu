@@ -341,14 +341,18 @@ mla_status_t mla_decode_plan(const int32_t *seq_lens, int batch, int q_len, int 
 
 }  // extern "C"
 
-// Validation and launch shared by the decode entry points; `cuda_cores`
-// selects the CUDA-core kernel (debug entry point) instead of the tensor-core one.
-static mla_status_t decode_entry(const mla_bf16_t *q_full, const mla_bf16_t *cache,
+// Validation and launch shared by the decode entry points: the tensor-core
+// kernel on the bf16 cache, the CUDA-core kernel (debug entry point), or the
+// tensor-core kernel on the FP8 cache (`fp8_scales` != NULL).
+enum DecodeKind { kTensorCore, kCudaCore, kTensorCoreFp8 };
+
+static mla_status_t decode_entry(const mla_bf16_t *q_full, const void *cache,
                                  int num_pages, const int32_t *block_table, int max_pages,
                                  int batch, int q_len, int n_h, float scale,
                                  const void *plan_host, const void *plan_dev, void *workspace,
                                  size_t workspace_bytes_given, mla_bf16_t *o_latent, float *lse,
-                                 uint32_t *status, mla_stream_t stream, bool cuda_cores) {
+                                 uint32_t *status, mla_stream_t stream, DecodeKind kind,
+                                 const float *fp8_scales = nullptr) {
   clear_error();
   MLA_CHECK_ARG(plan_host != nullptr && plan_dev != nullptr, "plan pointers are NULL");
   const PlanHeader *ph = static_cast<const PlanHeader *>(plan_host);
@@ -357,6 +361,8 @@ static mla_status_t decode_entry(const mla_bf16_t *q_full, const mla_bf16_t *cac
                 "plan was built for batch %d, q_len %d, n_h %d", ph->batch, ph->q_len, ph->n_h);
   if (batch == 0 || ph->num_items == 0) return MLA_OK;
   MLA_CHECK_ARG(q_full && cache && block_table && o_latent, "NULL device pointer");
+  MLA_CHECK_ARG(kind != kTensorCoreFp8 || (fp8_scales != nullptr && aligned16(fp8_scales)),
+                "the FP8 cache needs a 16-byte aligned scale array");
   MLA_CHECK_ARG(aligned16(q_full) && aligned16(cache) && aligned16(o_latent) &&
                     aligned16(plan_dev) && (workspace == nullptr || aligned16(workspace)),
                 "pointers must be 16-byte aligned");
@@ -373,7 +379,8 @@ static mla_status_t decode_entry(const mla_bf16_t *q_full, const mla_bf16_t *cac
   if (st != MLA_OK) return st;
   DecodeArgs a;
   a.q_full = q_full;
-  a.cache = cache;
+  a.cache = static_cast<const uint16_t *>(cache);
+  a.fp8_scales = fp8_scales;
   a.num_pages = num_pages;
   a.block_table = block_table;
   a.max_pages = max_pages;
@@ -390,8 +397,9 @@ static mla_status_t decode_entry(const mla_bf16_t *q_full, const mla_bf16_t *cac
   a.o_latent = o_latent;
   a.lse = lse;
   a.status = status;
-  st = cuda_cores ? launch_decode_simt(a, (cudaStream_t)stream)
-                  : launch_decode(a, (cudaStream_t)stream);
+  st = kind == kCudaCore ? launch_decode_simt(a, (cudaStream_t)stream)
+       : kind == kTensorCoreFp8 ? launch_decode_fp8(a, (cudaStream_t)stream)
+                                : launch_decode(a, (cudaStream_t)stream);
   if (st != MLA_OK) return st;
   return launch_combine(a, (cudaStream_t)stream);
 }
@@ -406,7 +414,7 @@ mla_status_t mla_decode_attention(const mla_bf16_t *q_full, const mla_bf16_t *ca
                                   uint32_t *status, mla_stream_t stream) {
   return decode_entry(q_full, cache, num_pages, block_table, max_pages, batch, q_len, n_h, scale,
                       plan_host, plan_dev, workspace, workspace_bytes_given, o_latent, lse,
-                      status, stream, false);
+                      status, stream, kTensorCore);
 }
 
 mla_status_t mla_decode_attention_cudacore(const mla_bf16_t *q_full, const mla_bf16_t *cache,
@@ -418,7 +426,44 @@ mla_status_t mla_decode_attention_cudacore(const mla_bf16_t *q_full, const mla_b
                                            float *lse, uint32_t *status, mla_stream_t stream) {
   return decode_entry(q_full, cache, num_pages, block_table, max_pages, batch, q_len, n_h, scale,
                       plan_host, plan_dev, workspace, workspace_bytes_given, o_latent, lse,
-                      status, stream, true);
+                      status, stream, kCudaCore);
+}
+
+mla_status_t mla_decode_attention_fp8(const mla_bf16_t *q_full, const uint8_t *cache,
+                                      const float *scales, int num_pages,
+                                      const int32_t *block_table, int max_pages, int batch,
+                                      int q_len, int n_h, float scale, const void *plan_host,
+                                      const void *plan_dev, void *workspace,
+                                      size_t workspace_bytes_given, mla_bf16_t *o_latent,
+                                      float *lse, uint32_t *status, mla_stream_t stream) {
+  return decode_entry(q_full, cache, num_pages, block_table, max_pages, batch, q_len, n_h, scale,
+                      plan_host, plan_dev, workspace, workspace_bytes_given, o_latent, lse,
+                      status, stream, kTensorCoreFp8, scales);
+}
+
+mla_status_t mla_cache_append_fp8(uint8_t *cache, float *scales, int num_pages,
+                                  const int32_t *block_table, int batch, int max_pages,
+                                  const int32_t *seq_idx, const int32_t *pos,
+                                  const mla_bf16_t *c_kv, int ld_c, const mla_bf16_t *k_pe,
+                                  int ld_k, const float *rope_table, int max_pos, int n_tokens,
+                                  uint32_t *status, mla_stream_t stream) {
+  clear_error();
+  MLA_CHECK_ARG(n_tokens >= 0, "n_tokens < 0");
+  if (n_tokens == 0) return MLA_OK;
+  MLA_CHECK_ARG(cache && scales && block_table && seq_idx && pos && c_kv && k_pe && rope_table,
+                "NULL device pointer");
+  MLA_CHECK_ARG(num_pages > 0 && batch > 0 && max_pages > 0 && max_pos > 0,
+                "sizes must be positive");
+  MLA_CHECK_ARG(aligned16(cache) && aligned16(scales) && aligned16(c_kv) && aligned16(k_pe) &&
+                    aligned16(rope_table),
+                "cache, scales, c_kv, k_pe and rope_table must be 16-byte aligned");
+  MLA_CHECK_ARG(ld_c >= MLA_D_C && ld_c % 8 == 0, "ld_c must be >= 512 and a multiple of 8");
+  MLA_CHECK_ARG(ld_k >= MLA_D_R && ld_k % 8 == 0, "ld_k must be >= 64 and a multiple of 8");
+  mla_status_t st = require_sm100();
+  if (st != MLA_OK) return st;
+  return launch_cache_append_fp8(cache, scales, num_pages, block_table, batch, max_pages, seq_idx,
+                                 pos, c_kv, ld_c, k_pe, ld_k, rope_table, max_pos, n_tokens,
+                                 status, (cudaStream_t)stream);
 }
 
 mla_status_t mla_debug_decode_wait(double wait_cap_seconds, int suppress_arrive) {

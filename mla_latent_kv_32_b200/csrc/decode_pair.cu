@@ -51,29 +51,30 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 320;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
+constexpr int kConvWarp0 = 10;                       // FP8 cache: converter warps 10..13
+constexpr int kConvWarps = 4;
+constexpr int kConvThreads = 32 * kConvWarps;
 constexpr int kTilePages = 4;                       // pages per score tile (256 tokens)
 constexpr int kChunksQK = MLA_ROW / 64;              // 9 column chunks of the score MMA
-constexpr int kStages = 7;
 constexpr uint32_t kBox = 64 * 128;                  // 64 rows x 64 bf16, 128-byte swizzle
 constexpr uint32_t kStageBytes = 2 * kBox;           // 16384
 constexpr uint32_t kOffQ = 0;                        // 9 x [64 heads][64 cols]
 constexpr uint32_t kOffP = kOffQ + kChunksQK * kBox; // 73728: 4 x [64 heads][64 tokens]
-constexpr uint32_t kOffRing = kOffP + kTilePages * kBox;            // 106496
-constexpr uint32_t kOffBar = kOffRing + kStages * kStageBytes;      // 221184
-constexpr uint32_t kOffPM = kOffBar + 256;           // row maxes [2 parity][4 pages][64]
-constexpr uint32_t kOffPL = kOffPM + 2 * 4 * 64 * 4; // row sums [4 pages][64]
-constexpr uint32_t kSmemUsed = kOffPL + 4 * 64 * 4;
-// The dynamic shared window of sm_100 starts 1024-byte aligned (after the
-// 1 KB reserved area); the kernel checks this and refuses to run otherwise.
-constexpr uint32_t kSmemBytes = kSmemUsed;
+constexpr uint32_t kOffRing = kOffP + kTilePages * kBox;  // 106496: bf16 operand stages
+constexpr uint32_t kLandStride = kBox + 1024;        // FP8 landing slot: 8 KB rows + scales
+constexpr uint32_t kBarArea = 384;
+
+constexpr int kMaxStages = 7;                        // capacity of the stage barrier arrays
+constexpr int kMaxLand = 9;                          // capacity of the landing barrier arrays
 
 enum {
-  B_FULL0 = 0,                     // [kStages] stage loaded (even CTA: both CTAs' bytes)
-  B_EMPTY0 = B_FULL0 + kStages,    // [kStages] stage consumed (both CTAs)
-  B_QFULL = B_EMPTY0 + kStages,    // query rows loaded (even CTA: both CTAs' bytes)
+  B_FULL0 = 0,                          // [kMaxStages] stage ready (even CTA)
+  B_EMPTY0 = B_FULL0 + kMaxStages,      // [kMaxStages] stage consumed (both CTAs)
+  B_LFULL0 = B_EMPTY0 + kMaxStages,     // [kMaxLand] FP8 landing slot loaded (local)
+  B_LEMPTY0 = B_LFULL0 + kMaxLand,      // [kMaxLand] FP8 landing slot converted (local)
+  B_QFULL = B_LEMPTY0 + kMaxLand,       // query rows loaded (even CTA: both CTAs' bytes)
   B_QEMPTY,                        // last score MMA of the item done (both)
   B_SFULL0, B_SFULL1,              // scores of a tile ready (both)
   B_SFREE0, B_SFREE1,              // scores read out (even CTA: 16 warps of both CTAs)
@@ -84,10 +85,28 @@ enum {
   B_FINAL,                         // MMA drain (even CTA)
   B_COUNT
 };
-constexpr uint32_t kOffTmemPtr = kOffBar + 8 * B_COUNT;
-constexpr uint32_t kOffAbort = kOffTmemPtr + 4;
-static_assert(kOffAbort + 4 <= kOffPM, "barrier area overflow");
-static_assert(kSmemBytes <= 232448, "shared memory budget");
+static_assert(8 * B_COUNT + 8 <= kBarArea, "barrier area overflow");
+
+// Shared-memory layout of the two instances. bf16 cache: a 7-stage ring of
+// bf16 operand stages filled by TMA. FP8 cache: a 4-stage ring of the same
+// bf16 stages, written by converter warps from a 6-slot ring of FP8 landing
+// slots (one page x 128 byte columns, plus the page's 64 token scales).
+template <bool kFp8>
+struct Cfg {
+  static constexpr int kThreads = kFp8 ? 32 * (kConvWarp0 + kConvWarps) : 320;
+  static constexpr int kStages = kFp8 ? 2 : 7;
+  static constexpr int kLand = kFp8 ? 9 : 0;
+  static constexpr uint32_t kOffLand = kOffRing + kStages * kStageBytes;
+  static constexpr uint32_t kOffBar = kOffLand + kLand * kLandStride;
+  static constexpr uint32_t kOffTmemPtr = kOffBar + 8 * B_COUNT;
+  static constexpr uint32_t kOffAbort = kOffTmemPtr + 4;
+  static constexpr uint32_t kOffPM = kOffBar + kBarArea;  // row maxes [2 parity][4 pages][64]
+  static constexpr uint32_t kOffPL = kOffPM + 2 * 4 * 64 * 4;  // row sums [4 pages][64]
+  static constexpr uint32_t kSmemBytes = kOffPL + 4 * 64 * 4;
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+  static_assert((kOffLand & 1023) == 0 && (kLandStride & 1023) == 0, "landing alignment");
+  static_assert(kStages <= kMaxStages && kLand <= kMaxLand, "barrier arrays too small");
+};
 
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemO = 0;      // [0, 256): output accumulator, chunk j at 128 j
@@ -106,14 +125,15 @@ struct PairArgs {
   uint32_t *status;
   uint64_t wait_ns;     // bound of every barrier wait
   int suppress_arrive;  // test hook: skip the first arrival on stage 0
+  const float *scales;  // FP8 cache: [num_pages][64] per-token scales
 };
 
 struct Ctx {
-  uint32_t base;
+  uint32_t bar_base;
   volatile int *abort_flag;
   uint32_t *status;
   uint64_t wait_ns;
-  __device__ uint32_t bar(int i) const { return base + kOffBar + 8u * i; }
+  __device__ uint32_t bar(int i) const { return bar_base + 8u * i; }
 };
 
 // Bounded wait on an mbarrier phase (acquire at cluster scope when `cluster`).
@@ -187,9 +207,44 @@ __device__ __forceinline__ uint32_t pack_hi_pair(uint32_t a_hi, uint32_t b_hi) {
 
 __device__ __forceinline__ int tiles_of(int np) { return (np + kTilePages - 1) / kTilePages; }
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+// E4M3 -> float by bit placement: the code's sign goes to bit 31 and its 7
+// exponent/mantissa bits to bits 26..20, which is the float 2^-120 times the
+// code's value for normal and subnormal codes alike (the E4M3 subnormal
+// 0.mmm x 2^-6 lands on the float subnormal 0.mmm x 2^-126). Multiplying by
+// 2^120 and then by the power-of-two scale is exact, and so is keeping the
+// upper 16 bits as the bf16 value (4 significant bits). Integer and FMA
+// pipes only.
+// 16 E4M3 codes (16 bytes, element 0 lowest) -> 16 bf16 values code * sc.
+__device__ __forceinline__ void fp8x16_to_bf16(const uint4 &v, float sc, uint4 &o0, uint4 &o1) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  const float k120 = 1.329227995784916e36f;   // 2^120
+  uint32_t r[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t x = w[i];
+    const uint32_t f0 = ((x << 24) & 0x80000000u) | ((x << 20) & 0x07F00000u);
+    const uint32_t f1 = ((x << 16) & 0x80000000u) | ((x << 12) & 0x07F00000u);
+    const uint32_t f2 = ((x << 8) & 0x80000000u) | ((x << 4) & 0x07F00000u);
+    const uint32_t f3 = (x & 0x80000000u) | ((x >> 4) & 0x07F00000u);
+    const float g0 = __uint_as_float(f0) * k120 * sc, g1 = __uint_as_float(f1) * k120 * sc;
+    const float g2 = __uint_as_float(f2) * k120 * sc, g3 = __uint_as_float(f3) * k120 * sc;
+    r[2 * i] = __byte_perm(__float_as_uint(g0), __float_as_uint(g1), 0x7632);
+    r[2 * i + 1] = __byte_perm(__float_as_uint(g2), __float_as_uint(g3), 0x7632);
+  }
+  o0 = make_uint4(r[0], r[1], r[2], r[3]);
+  o1 = make_uint4(r[4], r[5], r[6], r[7]);
+}
+
+template <bool kFp8>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<kFp8>::kThreads, 1)
 decode_pair_kernel(const __grid_constant__ CUtensorMap tm_cache,
                    const __grid_constant__ CUtensorMap tm_q, const PairArgs a) {
+  constexpr int kStages = Cfg<kFp8>::kStages;
+  constexpr int kLand = Cfg<kFp8>::kLand > 0 ? Cfg<kFp8>::kLand : 1;  // the bf16 instance has none
+  constexpr uint32_t kOffTmemPtr = Cfg<kFp8>::kOffTmemPtr;
+  constexpr uint32_t kOffAbort = Cfg<kFp8>::kOffAbort;
+  constexpr uint32_t kOffPM = Cfg<kFp8>::kOffPM;
+  constexpr uint32_t kOffPL = Cfg<kFp8>::kOffPL;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const uint32_t base = smem_u32(smem_raw);
   unsigned char *smem = smem_raw;
@@ -206,7 +261,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_cache,
   const int list = blockIdx.x >> 1;
 
   Ctx c;
-  c.base = base;
+  c.bar_base = base + Cfg<kFp8>::kOffBar;
   c.abort_flag = reinterpret_cast<volatile int *>(smem + kOffAbort);
   c.status = a.status;
   c.wait_ns = a.wait_ns;
@@ -214,8 +269,13 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_cache,
   if (threadIdx.x == 0) {
     *c.abort_flag = 0;
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(c.bar(B_FULL0 + i), 1);
+      // FP8: every converter warp of both CTAs arrives once per stage
+      mbar_init(c.bar(B_FULL0 + i), kFp8 ? 2 * kConvWarps : 1);
       mbar_init(c.bar(B_EMPTY0 + i), 1);
+    }
+    for (int i = 0; i < kLand; ++i) {
+      mbar_init(c.bar(B_LFULL0 + i), 1);
+      mbar_init(c.bar(B_LEMPTY0 + i), kConvWarps);
     }
     mbar_init(c.bar(B_QFULL), 1);
     mbar_init(c.bar(B_QEMPTY), 1);
@@ -244,11 +304,215 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_cache,
   const int i0 = cta_begin[list], i1 = cta_begin[list + 1];
 
   const uint32_t q_s = base + kOffQ, p_s = base + kOffP, ring = base + kOffRing;
+  const uint32_t land_s = base + Cfg<kFp8>::kOffLand;
   // barriers of the even CTA, as seen from this CTA
   const uint32_t lead_full0 = mapa_shared(c.bar(B_FULL0), 0);
   const uint32_t lead_qfull = mapa_shared(c.bar(B_QFULL), 0);
+  // page ids of tile t of an item: -2 for pages past the item's end; a bad id
+  // is reported and replaced by page 0 (loaded, then masked by the softmax)
+  auto tile_pages = [&](const WorkItem &wi, int t, bool check, int (&ids)[kTilePages]) {
+    const int32_t *row_pages = a.block_table + (size_t)wi.b * a.max_pages;
+#pragma unroll
+    for (int p = 0; p < kTilePages; ++p) {
+      const int pg = wi.page_begin + kTilePages * t + p;
+      int id = -2;
+      if (pg < wi.page_end) {
+        id = pg < a.max_pages ? row_pages[pg] : -1;
+        if (id < 0 || id >= a.num_pages) {
+          if (check) report(a.status, MLA_DEV_BAD_PAGE);
+          id = 0;
+        }
+      }
+      ids[p] = id;
+    }
+  };
 
-  if (warp == kProducerWarp) {
+  if (kFp8 && warp == kProducerWarp) {
+    // ---------------------------------------- FP8 landing producer ---
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_cache);
+      tma_prefetch_desc(&tm_q);
+      uint32_t lc = 0, ic = 0, q_armed = 0;
+      bool ok = true;
+      // one landing slot: 64 rows x 128 bytes of the page at byte column x
+      // (+ the page's 64 scales)
+      auto land = [&](int x, int id, bool with_scales) -> bool {
+        const uint32_t l = lc % kLand;
+        if (lc >= kLand && !wait_fast(c, c.bar(B_LEMPTY0 + l), ((lc / kLand) - 1) & 1, false))
+          return false;
+        const uint32_t dst = land_s + l * kLandStride;
+        mbar_arrive_expect_tx(c.bar(B_LFULL0 + l), kBox + (with_scales ? 256u : 0u));
+        tma_load_2d(dst, &tm_cache, x, id * 64, c.bar(B_LFULL0 + l));
+        if (with_scales) bulk_load(dst + kBox, a.scales + (size_t)id * 64, 256, c.bar(B_LFULL0 + l));
+        ++lc;
+        return true;
+      };
+      for (int it = i0; it < i1 && ok; ++it, ++ic) {
+        const WorkItem wi = items[it];
+        const int T = tiles_of(wi.page_end - wi.page_begin);
+        if (ic > 0 && !wait_bar(c, c.bar(B_QEMPTY), (ic - 1) & 1, false)) { ok = false; break; }
+        if (leader) {
+          mbar_arrive_expect_tx(c.bar(B_QFULL), 2 * kChunksQK * kBox);
+          ++q_armed;
+        }
+        const int tq = wi.b * a.q_len + wi.j;
+        for (int ch = 0; ch < kChunksQK; ++ch)
+          tma_load_3d_pair(q_s + ch * kBox, &tm_q, 64 * ch, 64 * (int)rank, tq, lead_qfull);
+        int ids_prev[kTilePages], ids_cur[kTilePages];
+        auto land_qk = [&](const int (&ids)[kTilePages]) -> bool {
+          for (int g = 0; g < 4; ++g)
+            for (int e = 0; e < 2; ++e)
+              if (ids[2 * rank + e] != -2 && !land(128 * g, ids[2 * rank + e], true)) return false;
+          for (int e = 0; e < 2; ++e)
+            if (ids[2 * rank + e] != -2 && !land(MLA_D_C, ids[2 * rank + e], false)) return false;
+          return true;
+        };
+        auto land_pv = [&](const int (&ids)[kTilePages]) -> bool {
+          for (int j = 0; j < 2; ++j)
+            for (int p = 0; p < kTilePages; ++p)
+              if (ids[p] != -2 && !land(128 * (2 * j + (int)rank), ids[p], true)) return false;
+          return true;
+        };
+        for (int t = 0; t < T && ok; ++t) {
+          tile_pages(wi, t, true, ids_cur);
+          if (!land_qk(ids_cur)) { ok = false; break; }
+          if (t >= 1 && !land_pv(ids_prev)) { ok = false; break; }
+#pragma unroll
+          for (int p = 0; p < kTilePages; ++p) ids_prev[p] = ids_cur[p];
+        }
+        if (ok && !land_pv(ids_prev)) ok = false;
+      }
+      // drain: every landing load completes on this CTA's own barriers
+      bool drained = true;
+      for (uint32_t k = lc > (uint32_t)kLand ? lc - kLand : 0; k < lc && drained; ++k)
+        drained = wait_drain(c, c.bar(B_LFULL0 + k % kLand), (k / kLand) & 1);
+      if (leader && q_armed && drained) wait_drain(c, c.bar(B_QFULL), (q_armed - 1) & 1);
+    }
+  } else if (kFp8 && warp >= kConvWarp0) {
+    // ------------------------------------------------ FP8 converters ---
+    // Walk the same stage sequence as the MMA issuer and the same landing
+    // sequence as the producer; write bf16 operand stages (128-byte
+    // swizzle) from the E4M3 landing slots, times each token's scale.
+    const int ci = threadIdx.x - 32 * kConvWarp0;   // 0..kConvThreads-1
+    const uint32_t lead_full = leader ? c.bar(B_FULL0) : lead_full0;
+    uint32_t sg = 0, lc = 0;
+    bool ok = true;
+    auto take_stage = [&](uint32_t &stg) -> bool {
+      stg = sg % kStages;
+      return sg < (uint32_t)kStages ||
+             wait_warp(c, c.bar(B_EMPTY0 + stg), ((sg / kStages) - 1) & 1, false);
+    };
+    auto give_stage = [&](uint32_t stg) {
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        if (leader)
+          mbar_arrive(lead_full + 8 * stg);
+        else
+          mbar_arrive_remote(lead_full + 8 * stg);
+      }
+      ++sg;
+    };
+    auto wait_land = [&](uint32_t k) {
+      return wait_warp(c, c.bar(B_LFULL0 + k % kLand), (k / kLand) & 1, false);
+    };
+    auto free_land = [&](uint32_t k) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(c.bar(B_LEMPTY0 + k % kLand));
+    };
+    auto slot = [&](uint32_t k) { return land_s + (k % kLand) * kLandStride - base; };
+    for (int it = i0; it < i1 && ok; ++it) {
+      const WorkItem wi = items[it];
+      const int T = tiles_of(wi.page_end - wi.page_begin);
+      int ids_prev[kTilePages], ids_cur[kTilePages];
+      auto conv_pv = [&](const int (&ids)[kTilePages]) -> bool {
+        for (int j = 0; j < 2; ++j)
+          for (int p = 0; p < kTilePages; ++p) {
+            if (ids[p] == -2) continue;
+            uint32_t stg;
+            if (!wait_land(lc) || !take_stage(stg)) return false;
+            const uint32_t src = slot(lc), dst = ring + stg * kStageBytes - base;
+            const float *sc = reinterpret_cast<const float *>(smem + src + kBox);
+#pragma unroll 4
+            for (int k = 0; k < 512 / kConvThreads; ++k) {
+              const int U = ci + kConvThreads * k, t = U >> 3, u = U & 7, sw = t & 7;
+              const uint4 v = *reinterpret_cast<const uint4 *>(smem + src + t * 128 + ((u ^ sw) << 4));
+              uint4 o0, o1;
+              fp8x16_to_bf16(v, sc[t], o0, o1);
+              unsigned char *row = smem + dst + (u >> 2) * kBox + t * 128;
+              const int lu = 2 * (u & 3);
+              *reinterpret_cast<uint4 *>(row + ((lu ^ sw) << 4)) = o0;
+              *reinterpret_cast<uint4 *>(row + (((lu + 1) ^ sw) << 4)) = o1;
+            }
+            give_stage(stg);
+            free_land(lc);
+            ++lc;
+          }
+        return true;
+      };
+      for (int t = 0; t < T && ok; ++t) {
+        tile_pages(wi, t, false, ids_cur);
+        const bool pres[2] = {ids_cur[2 * rank] != -2, ids_cur[2 * rank + 1] != -2};
+        // score chunks 2g, 2g+1 from group g of the CTA's two pages
+        for (int g = 0; g < 4 && ok; ++g) {
+          const uint32_t k0 = lc, k1 = lc + (pres[0] ? 1 : 0);
+          lc += (pres[0] ? 1 : 0) + (pres[1] ? 1 : 0);
+          if ((pres[0] && !wait_land(k0)) || (pres[1] && !wait_land(k1))) { ok = false; break; }
+          for (int h = 0; h < 2; ++h) {
+            uint32_t stg;
+            if (!take_stage(stg)) { ok = false; break; }
+            const uint32_t dst = ring + stg * kStageBytes - base;
+#pragma unroll 4
+            for (int k = 0; k < 512 / kConvThreads; ++k) {
+              const int U = ci + kConvThreads * k, e = U >> 8, t = (U >> 2) & 63, uu = U & 3,
+                        sw = t & 7;
+              if (!pres[e]) continue;
+              const uint32_t src = slot(e ? k1 : k0);
+              const int u = 4 * h + uu;
+              const uint4 v = *reinterpret_cast<const uint4 *>(smem + src + t * 128 + ((u ^ sw) << 4));
+              const float sc = reinterpret_cast<const float *>(smem + src + kBox)[t];
+              uint4 o0, o1;
+              fp8x16_to_bf16(v, sc, o0, o1);
+              unsigned char *row = smem + dst + e * kBox + t * 128;
+              *reinterpret_cast<uint4 *>(row + (((2 * uu) ^ sw) << 4)) = o0;
+              *reinterpret_cast<uint4 *>(row + (((2 * uu + 1) ^ sw) << 4)) = o1;
+            }
+            give_stage(stg);
+          }
+          if (!ok) break;
+          if (pres[0]) free_land(k0);
+          if (pres[1]) free_land(k1);
+        }
+        if (!ok) break;
+        // the RoPE chunk: bf16 rows copied unit by unit (same swizzle)
+        {
+          const uint32_t k0 = lc, k1 = lc + (pres[0] ? 1 : 0);
+          lc += (pres[0] ? 1 : 0) + (pres[1] ? 1 : 0);
+          uint32_t stg;
+          if ((pres[0] && !wait_land(k0)) || (pres[1] && !wait_land(k1)) || !take_stage(stg)) {
+            ok = false;
+            break;
+          }
+          const uint32_t dst = ring + stg * kStageBytes - base;
+#pragma unroll 4
+          for (int k = 0; k < 1024 / kConvThreads; ++k) {
+            const int U = ci + kConvThreads * k, e = U >> 9, t = (U >> 3) & 63, u = U & 7;
+            if (!pres[e]) continue;
+            const int off = t * 128 + ((u ^ (t & 7)) << 4);
+            *reinterpret_cast<uint4 *>(smem + dst + e * kBox + off) =
+                *reinterpret_cast<const uint4 *>(smem + slot(e ? k1 : k0) + off);
+          }
+          give_stage(stg);
+          if (pres[0]) free_land(k0);
+          if (pres[1]) free_land(k1);
+        }
+        if (t >= 1 && !conv_pv(ids_prev)) { ok = false; break; }
+#pragma unroll
+        for (int p = 0; p < kTilePages; ++p) ids_prev[p] = ids_cur[p];
+      }
+      if (ok && !conv_pv(ids_prev)) ok = false;
+    }
+  } else if (!kFp8 && warp == kProducerWarp) {
     if (lane == 0) {
       tma_prefetch_desc(&tm_cache);
       tma_prefetch_desc(&tm_q);
@@ -265,7 +529,6 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_cache,
         const WorkItem wi = items[it];
         const int np = wi.page_end - wi.page_begin;
         const int T = tiles_of(np);
-        const int32_t *row_pages = a.block_table + (size_t)wi.b * a.max_pages;
         if (ic > 0 && !wait_bar(c, c.bar(B_QEMPTY), (ic - 1) & 1, false)) { ok = false; break; }
         if (leader) {
           mbar_arrive_expect_tx(c.bar(B_QFULL), 2 * kChunksQK * kBox);
@@ -276,21 +539,6 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_cache,
           tma_load_3d_pair(q_s + ch * kBox, &tm_q, 64 * ch, 64 * (int)rank, tq, lead_qfull);
 
         int ids_prev[kTilePages], ids_cur[kTilePages];
-        auto fetch = [&](int t, int (&ids)[kTilePages]) {
-#pragma unroll
-          for (int p = 0; p < kTilePages; ++p) {
-            const int pg = wi.page_begin + kTilePages * t + p;
-            int id = -2;  // -2: no such page in this item
-            if (pg < wi.page_end) {
-              id = pg < a.max_pages ? row_pages[pg] : -1;
-              if (id < 0 || id >= a.num_pages) {
-                report(a.status, MLA_DEV_BAD_PAGE);
-                id = 0;  // load something valid; the softmax masks the page
-              }
-            }
-            ids[p] = id;
-          }
-        };
         auto load_qk = [&](const int (&ids)[kTilePages]) -> bool {
           int present = 0;
 #pragma unroll
@@ -332,7 +580,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_cache,
           return true;
         };
         for (int t = 0; t < T && ok; ++t) {
-          fetch(t, ids_cur);
+          tile_pages(wi, t, true, ids_cur);
           if (!load_qk(ids_cur)) { ok = false; break; }
           if (t >= 1 && !load_pv(ids_prev)) { ok = false; break; }
 #pragma unroll
@@ -426,7 +674,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_cache,
       mma_commit_pair_leader(c.bar(B_FINAL));
       wait_drain(c, c.bar(B_FINAL), 0);  // every MMA issued has completed
     }
-  } else {
+  } else if (warp < kProducerWarp) {
     // ------------------------------------------- softmax + epilogue warps ---
     const int q4 = warp & 3;                 // TMEM lane quarter
     const int grp = warp >> 2;               // column group
@@ -620,6 +868,8 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_cache,
   cluster_sync();
 }
 
+}  // namespace
+
 // ------------------------------------------------------------------ host ---
 
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
@@ -668,10 +918,8 @@ mla_status_t make_query_map(CUtensorMap *tm, const void *base, int T, int n_h) {
 }
 
 // failure-detection switch (mla_debug_decode_wait)
-uint64_t g_wait_ns = 1000000000ull;
-int g_suppress_arrive = 0;
-
-}  // namespace
+static uint64_t g_wait_ns = 1000000000ull;
+static int g_suppress_arrive = 0;
 
 mla_status_t set_decode_wait(double seconds, int suppress_arrive) {
   if (!(seconds > 0.0 && seconds <= 10.0))
@@ -681,11 +929,29 @@ mla_status_t set_decode_wait(double seconds, int suppress_arrive) {
   return MLA_OK;
 }
 
-mla_status_t launch_decode_pair(const DecodeArgs &a, cudaStream_t stream) {
+// FP8 cache pool [rows][640 bytes] as 64-row x 128-byte boxes, 128-byte
+// swizzle: latent byte columns [128 g, +128) or the bf16 k^R at byte 512.
+mla_status_t make_fp8_cache_map(CUtensorMap *tm, const void *base, uint64_t rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (enc == nullptr) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  cuuint64_t dims[2] = {(cuuint64_t)kFp8RowBytes, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)kFp8RowBytes};
+  cuuint32_t box[2] = {128, 64};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return MLA_OK;
+}
+
+template <bool kFp8>
+static mla_status_t launch_pair(const DecodeArgs &a, cudaStream_t stream) {
   const PlanHeader *ph = a.plan_host;
   if (ph->num_items == 0 || ph->num_ctas == 0) return MLA_OK;
   CUtensorMap tm_cache, tm_q;
-  mla_status_t st = make_cache_map(&tm_cache, a.cache, (uint64_t)a.num_pages * MLA_PAGE);
+  mla_status_t st = kFp8 ? make_fp8_cache_map(&tm_cache, a.cache, (uint64_t)a.num_pages * MLA_PAGE)
+                         : make_cache_map(&tm_cache, a.cache, (uint64_t)a.num_pages * MLA_PAGE);
   if (st != MLA_OK) return st;
   st = make_query_map(&tm_q, a.q_full, a.batch * a.q_len, a.n_h);
   if (st != MLA_OK) return st;
@@ -704,12 +970,34 @@ mla_status_t launch_decode_pair(const DecodeArgs &a, cudaStream_t stream) {
   t.status = a.status;
   t.wait_ns = g_wait_ns;
   t.suppress_arrive = g_suppress_arrive;
-  MLA_CUDA_TRY(cudaFuncSetAttribute(decode_pair_kernel,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    (int)kSmemBytes));
-  decode_pair_kernel<<<2 * ph->num_ctas, kThreads, kSmemBytes, stream>>>(tm_cache, tm_q, t);
-  MLA_LAUNCH_CHECK("decode_pair_kernel");
+  t.scales = a.fp8_scales;
+  // the shared-memory opt-in is a per-device attribute: set it once per device
+  static std::mutex mu;
+  static bool set[64] = {};
+  int dev = 0;
+  MLA_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return fail(MLA_ERR_UNSUPPORTED, "device index %d", dev);
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (!set[dev]) {
+      MLA_CUDA_TRY(cudaFuncSetAttribute(decode_pair_kernel<kFp8>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)Cfg<kFp8>::kSmemBytes));
+      set[dev] = true;
+    }
+  }
+  decode_pair_kernel<kFp8><<<2 * ph->num_ctas, Cfg<kFp8>::kThreads, Cfg<kFp8>::kSmemBytes,
+                             stream>>>(tm_cache, tm_q, t);
+  MLA_LAUNCH_CHECK(kFp8 ? "decode_pair_kernel<fp8>" : "decode_pair_kernel");
   return MLA_OK;
+}
+
+mla_status_t launch_decode_pair(const DecodeArgs &a, cudaStream_t stream) {
+  return launch_pair<false>(a, stream);
+}
+
+mla_status_t launch_decode_fp8(const DecodeArgs &a, cudaStream_t stream) {
+  return launch_pair<true>(a, stream);
 }
 
 }  // namespace mla

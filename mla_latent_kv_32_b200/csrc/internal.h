@@ -47,6 +47,15 @@ mla_status_t launch_cache_append(uint16_t *cache, int num_pages, const int32_t *
                                  int max_pos, int n_tokens, uint32_t *status,
                                  cudaStream_t stream);
 
+// FP8 cache: bytes per token row ([512 E4M3 | 64 bf16]) and the append.
+constexpr int kFp8RowBytes = MLA_D_C + 2 * MLA_D_R;   // 640
+mla_status_t launch_cache_append_fp8(uint8_t *cache, float *scales, int num_pages,
+                                     const int32_t *block_table, int batch, int max_pages,
+                                     const int32_t *seq_idx, const int32_t *pos,
+                                     const uint16_t *c_kv, int ld_c, const uint16_t *k_pe, int ld_k,
+                                     const float *rope_table, int max_pos, int n_tokens,
+                                     uint32_t *status, cudaStream_t stream);
+
 struct DecodeArgs {
   const uint16_t *q_full;
   const uint16_t *cache;
@@ -62,8 +71,10 @@ struct DecodeArgs {
   uint16_t *o_latent;
   float *lse;
   uint32_t *status;
+  const float *fp8_scales;  // FP8 cache only: [num_pages][64] per-token scales
 };
 mla_status_t launch_decode_simt(const DecodeArgs &a, cudaStream_t stream);
+mla_status_t launch_decode_fp8(const DecodeArgs &a, cudaStream_t stream);
 mla_status_t launch_decode_pair(const DecodeArgs &a, cudaStream_t stream);
 mla_status_t set_decode_wait(double seconds, int suppress_arrive);  // mla_debug_decode_wait
 mla_status_t launch_combine(const DecodeArgs &a, cudaStream_t stream);

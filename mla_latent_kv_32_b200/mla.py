@@ -77,6 +77,10 @@ SIGNATURES = {
     "mla_reset_status": (_I, [_P, _P]),
     "mla_plan_used_bytes": (_SZ, [_P]),
     "mla_plan_upload": (_I, [_P, _P, _SZ, _P]),
+    "mla_cache_append_fp8": (_I, [_P, _P, _I, _P, _I, _I, _P, _P, _P, _I, _P, _I, _P, _I, _I,
+                                  _P, _P]),
+    "mla_decode_attention_fp8": (_I, [_P, _P, _P, _I, _P, _I, _I, _I, _I, _F, _P, _P, _P, _SZ,
+                                      _P, _P, _P, _P]),
     "mla_fold_qk_workspace_bytes": (_SZ, [_I]),
     "mla_fold_qk": (_I, [_P, _I, _I, _P, _I, _P, _P, _SZ, _P]),
     "mla_fold_o": (_I, [_P, _I, _I, _P, _I, _P, _P]),
@@ -280,3 +284,23 @@ def mla_absorb_q_folded(x, ld_x, k_in, q_pe, ld_qp, w_qk, pos, rope_table, max_p
                                       _ptr(pos), _ptr(rope_table), max_pos, T, n_h,
                                       _ptr(q_full), _ptr(status), _stream(stream)),
            "mla_absorb_q_folded")
+
+
+def mla_cache_append_fp8(cache, scales, num_pages, block_table, batch, max_pages, seq_idx, pos,
+                         c_kv, ld_c, k_pe, ld_k, rope_table, max_pos, n_tokens, status=None,
+                         stream=None):
+    _check(load().mla_cache_append_fp8(_ptr(cache), _ptr(scales), num_pages, _ptr(block_table),
+                                       batch, max_pages, _ptr(seq_idx), _ptr(pos), _ptr(c_kv),
+                                       ld_c, _ptr(k_pe), ld_k, _ptr(rope_table), max_pos, n_tokens,
+                                       _ptr(status), _stream(stream)), "mla_cache_append_fp8")
+
+
+def mla_decode_attention_fp8(q_full, cache, scales, num_pages, block_table, max_pages, batch,
+                             q_len, n_h, scale, plan_host, plan_dev, workspace, workspace_bytes,
+                             o_latent, lse=None, status=None, stream=None):
+    _check(load().mla_decode_attention_fp8(_ptr(q_full), _ptr(cache), _ptr(scales), num_pages,
+                                           _ptr(block_table), max_pages, batch, q_len, n_h,
+                                           scale, _ptr(plan_host), _ptr(plan_dev),
+                                           _ptr(workspace), workspace_bytes, _ptr(o_latent),
+                                           _ptr(lse), _ptr(status), _stream(stream)),
+           "mla_decode_attention_fp8")

@@ -18,6 +18,8 @@ from . import mla
 
 D_C, D_R, D_NOPE, D_V, ROW, PAGE = mla.D_C, mla.D_R, mla.D_NOPE, mla.D_V, mla.ROW, mla.PAGE
 DEFAULT_SCALE = 1.0 / math.sqrt(D_NOPE + D_R)
+FP8_ROW = D_C + 2 * D_R      # bytes per FP8 cache row: [512 E4M3 | 64 bf16]
+FP8_FILL_CODE = 0x70         # E4M3 128.0: the filler of slots that hold no token
 
 
 def to_dev_bf16(bits: np.ndarray, device) -> torch.Tensor:
@@ -65,9 +67,11 @@ class DecodeSession(_GraphStep):
     """
 
     def __init__(self, inp, device="cuda", num_ctas: int = 0, max_split: int = -1,
-                 scale: float = DEFAULT_SCALE, rope_table: Optional[np.ndarray] = None):
+                 scale: float = DEFAULT_SCALE, rope_table: Optional[np.ndarray] = None,
+                 fp8: bool = False):
         w = inp.w
         self.w = w
+        self.fp8 = fp8
         self.device = torch.device(device)
         self.B, self.q_len, self.n_h = w.B, w.q_len, w.n_h
         self.T = w.B * w.q_len
@@ -76,7 +80,7 @@ class DecodeSession(_GraphStep):
         self.lens = inp.lens
         self.num_pages = inp.pool.shape[0]
         self.max_pages = inp.table.shape[1]
-        self.cache = to_dev_bf16(inp.pool, dev)
+        self.cache = None if fp8 else to_dev_bf16(inp.pool, dev)
         self.table = to_dev(inp.table, dev)
         self.q_nope = to_dev_bf16(inp.q_nope.reshape(self.T, -1), dev)
         self.q_pe = to_dev_bf16(inp.q_pe.reshape(self.T, -1), dev)
@@ -101,9 +105,48 @@ class DecodeSession(_GraphStep):
         self.lse = torch.empty((self.T, self.n_h), dtype=torch.float32, device=dev)
         self.u = torch.empty((self.T, self.n_h * D_V), dtype=torch.bfloat16, device=dev)
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        if fp8:
+            self._fp8_pool(inp)
+
+    def _fp8_pool(self, inp):
+        """The FP8 cache of this workload: every slot starts as a large
+        finite filler (latent code 128.0, scale 1, k^R bf16 64.0); the
+        workload's prefix rows [c | k] then enter through the library's own
+        FP8 append at their positions (k rotated there), as a prefill would
+        write them. The bf16 pool is dropped."""
+        dev = self.device
+        self.cache = None
+        self.cache8 = torch.empty((self.num_pages, PAGE, FP8_ROW), dtype=torch.uint8, device=dev)
+        self.cache8[:, :, :D_C] = FP8_FILL_CODE
+        self.cache8[:, :, D_C:].view(torch.int16).fill_(int(np.uint16(0x4280).view(np.int16)))
+        self.scales8 = torch.ones((self.num_pages, PAGE), dtype=torch.float32, device=dev)
+        table = inp.table
+        rows, seq, pos = [], [], []
+        for b in range(self.B):
+            n = int(inp.lens[b]) - self.q_len
+            if n <= 0:
+                continue
+            pages = table[b, :(n + PAGE - 1) // PAGE]
+            rows.append(inp.pool[pages].reshape(-1, ROW)[:n])
+            seq.append(np.full(n, b, np.int32))
+            pos.append(np.arange(n, dtype=np.int32))
+        if rows:
+            r = to_dev_bf16(np.concatenate(rows), dev)
+            sq, ps = to_dev(np.concatenate(seq), dev), to_dev(np.concatenate(pos), dev)
+            mla.mla_cache_append_fp8(self.cache8, self.scales8, self.num_pages, self.table, self.B,
+                                     self.max_pages, sq, ps, r, ROW, r[:, D_C:], ROW, self.rope,
+                                     self.max_pos, r.shape[0], self.status)
+            torch.cuda.synchronize(dev)
+            del r, sq, ps
 
     # the four calls of one step ------------------------------------------
     def append(self, stream=None):
+        if self.fp8:
+            mla.mla_cache_append_fp8(self.cache8, self.scales8, self.num_pages, self.table,
+                                     self.B, self.max_pages, self.seq_idx, self.pos, self.c_new,
+                                     D_C, self.k_new, D_R, self.rope, self.max_pos, self.T,
+                                     self.status, stream)
+            return
         mla.mla_cache_append(self.cache, self.num_pages, self.table, self.B, self.max_pages,
                              self.seq_idx, self.pos, self.c_new, D_C, self.k_new, D_R, self.rope,
                              self.max_pos, self.T, self.status, stream)
@@ -114,6 +157,13 @@ class DecodeSession(_GraphStep):
                          self.status, stream)
 
     def attend(self, stream=None, lse=True):
+        if self.fp8:
+            mla.mla_decode_attention_fp8(self.q_full, self.cache8, self.scales8, self.num_pages,
+                                         self.table, self.max_pages, self.B, self.q_len,
+                                         self.n_h, self.scale, self.plan_host, self.plan_dev,
+                                         self.workspace, self.ws_bytes, self.o,
+                                         self.lse if lse else None, self.status, stream)
+            return
         mla.mla_decode_attention(self.q_full, self.cache, self.num_pages, self.table,
                                  self.max_pages, self.B, self.q_len, self.n_h, self.scale,
                                  self.plan_host, self.plan_dev, self.workspace, self.ws_bytes,
