@@ -67,6 +67,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--workload", default="v3")
+    ap.add_argument("--cache", default="bf16", choices=["bf16", "fp8"],
+                    help="latent cache format of the timed workload")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the workload's batch (a smaller case of the same "
                          "workload, e.g. for profiling)")
@@ -613,7 +615,8 @@ def main():
         w = dataclasses.replace(w, B=args.batch)
     assert not w.layer, "bench.py times the attention-only decode workloads"
     inp = synth.make_decode_inputs(w)
-    sess = DecodeSession(inp, dev, num_ctas=args.num_ctas, max_split=args.max_split)
+    fp8 = args.cache == "fp8"
+    sess = DecodeSession(inp, dev, num_ctas=args.num_ctas, max_split=args.max_split, fp8=fp8)
     flush = L2Flush(dev)
     stream = torch.cuda.current_stream()
     peaks, peak_src = load_peaks()
@@ -667,6 +670,8 @@ def main():
         tokens = w.B * w.q_len
         value = whole_job_rate(world, tokens, t_step)
         cache_bytes, flops = attention_work(inp, w)
+        if fp8:
+            cache_bytes = int(inp.lens.sum()) * FP8_TOKEN_BYTES
 
         # e2e: per-step inputs uploaded from pinned host memory and the result
         # read back to pinned host memory, through the library's calls. Two
@@ -677,7 +682,8 @@ def main():
         # flush runs in this loop.
         e2e = None
         if not args.no_e2e:
-            sess2 = DecodeSession(inp, dev, num_ctas=args.num_ctas, max_split=args.max_split)
+            sess2 = DecodeSession(inp, dev, num_ctas=args.num_ctas, max_split=args.max_split,
+                                  fp8=fp8)
             pair = [sess, sess2]
             ins, host_in, host_out0 = sess.pinned_step_buffers()
             host_outs = [host_out0, torch.empty_like(host_out0).pin_memory()]
@@ -758,6 +764,7 @@ def main():
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": t_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "cache": "FP8 (E4M3 latent, bf16 k^R, per-token scale)" if fp8 else "bf16",
         "config": workload_config(w, inp, sess, args.ramp_seconds),
         "cache_gbs": cache_bytes / (t_step / 1e3) / 1e9 * world,
         "attention_ms": t_attn,

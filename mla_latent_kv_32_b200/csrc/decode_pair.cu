@@ -420,7 +420,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_cache,
       __syncwarp();
       if (lane == 0) mbar_arrive(c.bar(B_LEMPTY0 + k % kLand));
     };
-    auto slot = [&](uint32_t k) { return land_s + (k % kLand) * kLandStride - base; };
+    auto slot = [&](uint32_t k) { return land_s + (k % kLand) * kLandStride; };
     for (int it = i0; it < i1 && ok; ++it) {
       const WorkItem wi = items[it];
       const int T = tiles_of(wi.page_end - wi.page_begin);
@@ -431,18 +431,17 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_cache,
             if (ids[p] == -2) continue;
             uint32_t stg;
             if (!wait_land(lc) || !take_stage(stg)) return false;
-            const uint32_t src = slot(lc), dst = ring + stg * kStageBytes - base;
-            const float *sc = reinterpret_cast<const float *>(smem + src + kBox);
+            const uint32_t src = slot(lc), dst = ring + stg * kStageBytes;
 #pragma unroll 4
             for (int k = 0; k < 512 / kConvThreads; ++k) {
               const int U = ci + kConvThreads * k, t = U >> 3, u = U & 7, sw = t & 7;
-              const uint4 v = *reinterpret_cast<const uint4 *>(smem + src + t * 128 + ((u ^ sw) << 4));
+              const uint4 v = lds128(src + t * 128 + ((u ^ sw) << 4));
               uint4 o0, o1;
-              fp8x16_to_bf16(v, sc[t], o0, o1);
-              unsigned char *row = smem + dst + (u >> 2) * kBox + t * 128;
+              fp8x16_to_bf16(v, lds_f32(src + kBox + 4 * t), o0, o1);
+              const uint32_t row = dst + (u >> 2) * kBox + t * 128;
               const int lu = 2 * (u & 3);
-              *reinterpret_cast<uint4 *>(row + ((lu ^ sw) << 4)) = o0;
-              *reinterpret_cast<uint4 *>(row + (((lu + 1) ^ sw) << 4)) = o1;
+              sts128(row + ((lu ^ sw) << 4), o0);
+              sts128(row + (((lu + 1) ^ sw) << 4), o1);
             }
             give_stage(stg);
             free_land(lc);
@@ -461,7 +460,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_cache,
           for (int h = 0; h < 2; ++h) {
             uint32_t stg;
             if (!take_stage(stg)) { ok = false; break; }
-            const uint32_t dst = ring + stg * kStageBytes - base;
+            const uint32_t dst = ring + stg * kStageBytes;
 #pragma unroll 4
             for (int k = 0; k < 512 / kConvThreads; ++k) {
               const int U = ci + kConvThreads * k, e = U >> 8, t = (U >> 2) & 63, uu = U & 3,
@@ -469,13 +468,12 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_cache,
               if (!pres[e]) continue;
               const uint32_t src = slot(e ? k1 : k0);
               const int u = 4 * h + uu;
-              const uint4 v = *reinterpret_cast<const uint4 *>(smem + src + t * 128 + ((u ^ sw) << 4));
-              const float sc = reinterpret_cast<const float *>(smem + src + kBox)[t];
+              const uint4 v = lds128(src + t * 128 + ((u ^ sw) << 4));
               uint4 o0, o1;
-              fp8x16_to_bf16(v, sc, o0, o1);
-              unsigned char *row = smem + dst + e * kBox + t * 128;
-              *reinterpret_cast<uint4 *>(row + (((2 * uu) ^ sw) << 4)) = o0;
-              *reinterpret_cast<uint4 *>(row + (((2 * uu + 1) ^ sw) << 4)) = o1;
+              fp8x16_to_bf16(v, lds_f32(src + kBox + 4 * t), o0, o1);
+              const uint32_t row = dst + e * kBox + t * 128;
+              sts128(row + (((2 * uu) ^ sw) << 4), o0);
+              sts128(row + (((2 * uu + 1) ^ sw) << 4), o1);
             }
             give_stage(stg);
           }
@@ -493,14 +491,13 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_cache,
             ok = false;
             break;
           }
-          const uint32_t dst = ring + stg * kStageBytes - base;
+          const uint32_t dst = ring + stg * kStageBytes;
 #pragma unroll 4
           for (int k = 0; k < 1024 / kConvThreads; ++k) {
             const int U = ci + kConvThreads * k, e = U >> 9, t = (U >> 3) & 63, u = U & 7;
             if (!pres[e]) continue;
             const int off = t * 128 + ((u ^ (t & 7)) << 4);
-            *reinterpret_cast<uint4 *>(smem + dst + e * kBox + off) =
-                *reinterpret_cast<const uint4 *>(smem + slot(e ? k1 : k0) + off);
+            sts128(dst + e * kBox + off, lds128(slot(e ? k1 : k0) + off));
           }
           give_stage(stg);
           if (pres[0]) free_land(k0);
