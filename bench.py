@@ -56,7 +56,7 @@ def dist_stats(xs):
 # decode sources it was measured on and the workload; reported only while the
 # sources match (the combine kernel's few MB are not included).
 TRAFFIC = {
-    ("376d5e91cc46aef1", "v3"): 318149120,   # decode_pair_kernel
+    ("79c6a9d1edad444d", "v3"): 317488384,   # decode_pair_kernel<bf16>, 1.051 x the cache bytes
 }
 
 
@@ -707,8 +707,24 @@ def main():
             (t_e2e,) = max_over_ranks([t_e2e], dist, dev, world)
             for s_ in pair:
                 assert s_.read_status() == 0, "device status in the end-to-end loop"
+            # the host link alone: the same per-step copies timed by themselves
+            def copy_ms(fn, n=20):
+                a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                fn()
+                a_.record(stream)
+                for _ in range(n):
+                    fn()
+                b_.record(stream)
+                torch.cuda.synchronize()
+                return a_.elapsed_time(b_) / n
+
+            dev_in = sess.io_inputs()
+            t_h2d = copy_ms(lambda: [d.copy_(h_, non_blocking=True) for d, h_ in zip(dev_in, host_in)])
+            t_d2h = copy_ms(lambda: host_outs[0].copy_(sess.u, non_blocking=True))
             e2e = {"value": whole_job_rate(world, tokens, t_e2e), "unit": UNIT,
                    "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                   "host_link": {"h2d_ms": t_h2d, "d2h_ms": t_d2h,
+                                 "h2d_gbs": h2d / t_h2d / 1e6, "d2h_gbs": d2h / t_d2h / 1e6},
                    "ms_per_step": t_e2e, "steps": E,
                    "host_enqueue_us_per_step": host_s / E * 1e6,
                    "method": "two sessions, each one CUDA graph of upload (pinned host -> "
