@@ -88,6 +88,8 @@ def parse():
     ap.add_argument("--ramp-seconds", type=float, default=0.3,
                     help="back-to-back untimed steps before timing, so the clocks leave "
                          "their idle state (0: none, e.g. under a profiler)")
+    ap.add_argument("--rows-only", default="",
+                    help="with --rows: comma-separated row names to run (e.g. a1,a9)")
     ap.add_argument("--rows", action="store_true",
                     help="time every library call of the decode step (v3) and of the "
                          "full layer (layer_v3) alone against its own roofline; one JSON "
@@ -378,6 +380,11 @@ def run_rows(args):
             ts.append(a.elapsed_time(b) * 1e3)
         return statistics.median(ts)
 
+    only = {r for r in args.rows_only.split(",") if r}
+
+    def want(row):
+        return not only or row in only
+
     def line(workload, row, call, us, nbytes, flops):
         t_mem = nbytes / (peaks["hbm_gbs"] * 1e9) * 1e6
         t_tc = flops / (peaks["bf16_tflops"] * 1e12) * 1e6
@@ -392,39 +399,51 @@ def run_rows(args):
     K = max(5, args.steps)
     bf = 2
     # decode step rows on v3
-    w = synth.WORKLOADS["v3"]
-    inp = synth.make_decode_inputs(w)
-    sess = DecodeSession(inp, dev)
-    T, H = w.B * w.q_len, w.n_h
-    line("v3", "a3+a4", "mla_cache_append", timed(sess.append, K),
-         T * (576 * bf + 1152 + 256), 0)
-    line("v3", "a3+a5", "mla_absorb_q", timed(sess.absorb, K),
-         H * 128 * 512 * bf + T * H * (128 + 64 + 576) * bf + T * 256, 2.0 * T * H * 128 * 512)
-    cache = int(inp.lens.sum()) * ROW_BYTES
-    vis = sum(int(L) - w.q_len + j + 1 for L in inp.lens for j in range(w.q_len))
-    line("v3", "a6+a7", "mla_decode_attention", timed(sess.attend, K), cache,
-         float(vis) * H * FLOP_PER_TOKEN_HEAD)
-    line("v3", "a8", "mla_out_absorb", timed(sess.expand, K),
-         H * 128 * 512 * bf + T * H * (512 + 128) * bf, 2.0 * T * H * 128 * 512)
-    del sess, inp
-    torch.cuda.empty_cache()
+    if any(want(r) for r in ("a3+a4", "a3+a5", "a6+a7", "a8")):
+        w = synth.WORKLOADS["v3"]
+        inp = synth.make_decode_inputs(w)
+        sess = DecodeSession(inp, dev)
+        T, H = w.B * w.q_len, w.n_h
+        if want("a3+a4"):
+            line("v3", "a3+a4", "mla_cache_append", timed(sess.append, K),
+                 T * (576 * bf + 1152 + 256), 0)
+        if want("a3+a5"):
+            line("v3", "a3+a5", "mla_absorb_q", timed(sess.absorb, K),
+                 H * 128 * 512 * bf + T * H * (128 + 64 + 576) * bf + T * 256,
+                 2.0 * T * H * 128 * 512)
+        cache = int(inp.lens.sum()) * ROW_BYTES
+        vis = sum(int(L) - w.q_len + j + 1 for L in inp.lens for j in range(w.q_len))
+        if want("a6+a7"):
+            line("v3", "a6+a7", "mla_decode_attention", timed(sess.attend, K), cache,
+                 float(vis) * H * FLOP_PER_TOKEN_HEAD)
+        if want("a8"):
+            line("v3", "a8", "mla_out_absorb", timed(sess.expand, K),
+                 H * 128 * 512 * bf + T * H * (512 + 128) * bf, 2.0 * T * H * 128 * 512)
+        del sess, inp
+        torch.cuda.empty_cache()
+    if not any(want(r) for r in ("a1", "a2", "a6+a7", "a9")):
+        return 0
     # the whole layer's projections on layer_v3
     w = synth.WORKLOADS["layer_v3"]
     inp = synth.make_layer_inputs(w)
     ls = LayerSession(inp, dev)
     Tq, Tk, H, d, ql = ls.Tq, ls.T, w.n_h, w.hidden, w.q_lora
     nq = H * 192
-    line("layer_v3", "a1", "mla_gemm_bf16 x2 (W_DQ, [W_UQ|W_QR])", timed(ls.project_q, K),
-         (ql * d + Tq * d + Tq * ql) * bf + (nq * ql + Tq * ql + Tq * nq) * bf,
-         2.0 * Tq * ql * d + 2.0 * Tq * nq * ql)
-    line("layer_v3", "a2", "mla_gemm_bf16 ([W_DKV|W_KR])", timed(ls.project_kv, K),
-         (576 * d + Tk * d + Tk * 576) * bf, 2.0 * Tk * 576 * d)
+    if want("a1"):
+        line("layer_v3", "a1", "mla_gemm_bf16 x2 (W_DQ, [W_UQ|W_QR])", timed(ls.project_q, K),
+             (ql * d + Tq * d + Tq * ql) * bf + (nq * ql + Tq * ql + Tq * nq) * bf,
+             2.0 * Tq * ql * d + 2.0 * Tq * nq * ql)
+    if want("a2"):
+        line("layer_v3", "a2", "mla_gemm_bf16 ([W_DKV|W_KR])", timed(ls.project_kv, K),
+             (576 * d + Tk * d + Tk * 576) * bf, 2.0 * Tk * 576 * d)
     ls.project_q(); ls.project_kv(); ls.append(); ls.absorb()
-    line("layer_v3", "a6+a7", "mla_decode_attention", timed(ls.attend, K),
-         int(ls.lens.sum()) * ROW_BYTES,
-         float(sum(int(L) for L in ls.lens)) * H * FLOP_PER_TOKEN_HEAD)
-    line("layer_v3", "a9", "mla_gemm_bf16 (W_O, fp32 out)", timed(ls.project_out, K),
-         (d * H * 128 + Tq * H * 128) * bf + Tq * d * 4, 2.0 * Tq * d * H * 128)
+    if want("a6+a7"):
+        line("layer_v3", "a6+a7", "mla_decode_attention", timed(ls.attend, K),
+             int(ls.lens.sum()) * ROW_BYTES,
+             float(sum(int(L) for L in ls.lens)) * H * FLOP_PER_TOKEN_HEAD)
+    if want("a9"):
+        line("layer_v3", "a9", "mla_gemm_bf16 (W_O, fp32 out)", timed(ls.project_out, K),
+             (d * H * 128 + Tq * H * 128) * bf + Tq * d * 4, 2.0 * Tq * d * H * 128)
     return 0
 
 
@@ -497,7 +516,7 @@ def measure_decode_config(name, dev, flush, stream, K, peaks, args, fp8=False):
            "plan": {"work_lists": int(sess.info.num_ctas), "items": int(sess.info.num_items),
                     "partials": int(sess.info.num_partials),
                     "combine": int(sess.info.num_combine)},
-           "launches_per_step": 4 + (1 if sess.info.num_combine else 0)}
+           "launches_per_step": (4 if fp8 else 3) + (1 if sess.info.num_combine else 0)}
     if w.q_len > 16:
         # the same attention in the expanded (non-absorbed) form: 2*(128+64)
         # + 2*128 FLOP per (visible token, head, query) plus expanding K^C and
@@ -560,8 +579,7 @@ def measure_layer_config(name, dev, flush, stream, K, peaks, folded=False):
                            if folded else "")),
            "weight_bytes": wbytes,
            "tokens_per_s": Tq / (t_step / 1e3), "step_ms": t_step, "attention_ms": t_attn,
-           "step_ms_stats": dist_stats(step), "attention_ms_stats": dist_stats(attn),
-           "launches_per_step": (6 if folded else 7) + (1 if ls.info.num_combine else 0)}
+           "step_ms_stats": dist_stats(step), "attention_ms_stats": dist_stats(attn)}
     if big:
         out["l2"] = "flushed before every timed call"
         out["roofline_attention"] = roofline_of(cache_bytes, attn_flops, t_attn, peaks)
@@ -771,11 +789,12 @@ def main():
         "peak_source": f"{peak_src} (MEASURED_PEAKS.json burst figures)"
         if peak_src == "measured" else "fallback", "sources": src_hash,
     }
-    # cache_append, absorb GEMM (with the q RoPE pack in the same launch),
-    # decode, [combine], out_absorb per timed step, plus decode [+ combine]
-    # per timed attention call
+    # the absorb GEMM (with the q RoPE pack and the cache append in the same
+    # launch; the FP8 cache appends in its own launch), decode, [combine],
+    # out_absorb per timed step, plus decode [+ combine] per timed attention call
     combine = 1 if sess.info.num_combine > 0 else 0
-    launches_timed = K * (4 + combine) + K * (1 + combine)
+    per_step = (4 if fp8 else 3) + combine
+    launches_timed = K * per_step + K * (1 + combine)
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": t_step, "higher_is_better": True,

@@ -139,6 +139,25 @@ mla_status_t mla_absorb_q(const mla_bf16_t *q_nope, int ld_qn,
                           mla_bf16_t *q_full, uint32_t *status, mla_stream_t stream);
 
 /*
+ * mla_append_absorb_q -- device. mla_cache_append and mla_absorb_q of one
+ * decode step in one launch (the append runs in extra CTAs of the absorption
+ * GEMM, beside the q^R RoPE pack): the same results as the two calls in that
+ * order ("DeepSeek-V3 MLA ... Guide", "Step 3": append the new rows, absorb
+ * the query). The cache arguments are those of mla_cache_append (positions
+ * tok_pos, n_tokens rows), the query arguments those of mla_absorb_q
+ * (positions q_pos, may be NULL); the RoPE table is shared and required.
+ * The appended rows are not read by this call. Errors: as the two calls.
+ */
+mla_status_t mla_append_absorb_q(mla_bf16_t *cache, int num_pages, const int32_t *block_table,
+                                 int batch, int max_pages, const int32_t *seq_idx,
+                                 const int32_t *tok_pos, const mla_bf16_t *c_kv, int ld_c,
+                                 const mla_bf16_t *k_pe, int ld_k, int n_tokens,
+                                 const mla_bf16_t *q_nope, int ld_qn, const mla_bf16_t *q_pe,
+                                 int ld_qp, const mla_bf16_t *w_uk, const int32_t *q_pos,
+                                 const float *rope_table, int max_pos, int T, int n_h,
+                                 mla_bf16_t *q_full, uint32_t *status, mla_stream_t stream);
+
+/*
  * Decode plan. The split of each sequence's pages into work items is made on
  * the host from the sequence lengths (split-KV: long sequences are cut into
  * several items whose partial results are merged by a log-sum-exp combine).
@@ -330,14 +349,19 @@ mla_status_t mla_gemm_bf16(const mla_bf16_t *X, int ld_x, const mla_bf16_t *W, i
                            mla_stream_t stream);
 
 /*
- * mla_gemm_bf16_ws -- device. mla_gemm_bf16 with a caller workspace for
- * bf16 outputs: when the output has few 128 x 256 tiles and K is long (the
- * down-projections from the 7168-wide hidden state), the reduction is split
- * over K across more CTAs, fp32 partial sums accumulate in the workspace
- * (zeroed by the call) and one more kernel rounds them to bf16 into C. Same
- * result as mla_gemm_bf16 up to the order of the fp32 additions.
+ * mla_gemm_bf16_ws -- device. mla_gemm_bf16 with a caller workspace: when
+ * the output has few tiles and K is long (the down-projections from the
+ * 7168-wide hidden state, the output projection), the reduction is split over
+ * K across more CTAs. For a bf16 output the fp32 sums accumulate in the
+ * workspace (zeroed by the call) and one more kernel rounds them to bf16 into
+ * C; for an fp32 output each split writes its own partial tile into the
+ * workspace (no atomics, so the result does not depend on the order the CTAs
+ * finish in) and one more kernel adds them into C. Same result as
+ * mla_gemm_bf16 up to the order of the fp32 additions.
  *   workspace: device, 16-byte aligned, >= mla_gemm_bf16_workspace_bytes(M,
- *              N, K) bytes, or NULL (then exactly mla_gemm_bf16).
+ *              N, K) bytes (the larger of the two uses; it depends on the
+ *              current device's SM count), or NULL (then exactly
+ *              mla_gemm_bf16).
  * The workspace must not be in use by another call running at the same time.
  */
 size_t mla_gemm_bf16_workspace_bytes(int M, int N, int K);

@@ -153,6 +153,58 @@ mla_status_t mla_absorb_q(const mla_bf16_t *q_nope, int ld_qn, const mla_bf16_t 
                          q_full, status, (cudaStream_t)stream);
 }
 
+mla_status_t mla_append_absorb_q(mla_bf16_t *cache, int num_pages, const int32_t *block_table,
+                                 int batch, int max_pages, const int32_t *seq_idx,
+                                 const int32_t *tok_pos, const mla_bf16_t *c_kv, int ld_c,
+                                 const mla_bf16_t *k_pe, int ld_k, int n_tokens,
+                                 const mla_bf16_t *q_nope, int ld_qn, const mla_bf16_t *q_pe,
+                                 int ld_qp, const mla_bf16_t *w_uk, const int32_t *q_pos,
+                                 const float *rope_table, int max_pos, int T, int n_h,
+                                 mla_bf16_t *q_full, uint32_t *status, mla_stream_t stream) {
+  clear_error();
+  MLA_CHECK_ARG(n_tokens >= 0 && T >= 0, "negative size");
+  if (T == 0)
+    return mla_cache_append(cache, num_pages, block_table, batch, max_pages, seq_idx, tok_pos,
+                            c_kv, ld_c, k_pe, ld_k, rope_table, max_pos, n_tokens, status, stream);
+  if (n_tokens == 0)
+    return mla_absorb_q(q_nope, ld_qn, q_pe, ld_qp, w_uk, q_pos, rope_table, max_pos, T, n_h,
+                        q_full, status, stream);
+  // the append's arguments, as mla_cache_append checks them
+  MLA_CHECK_ARG(cache && block_table && seq_idx && tok_pos && c_kv && k_pe && rope_table,
+                "NULL device pointer");
+  MLA_CHECK_ARG(num_pages > 0 && batch > 0 && max_pages > 0 && max_pos > 0,
+                "sizes must be positive");
+  MLA_CHECK_ARG(aligned16(cache) && aligned16(c_kv) && aligned16(k_pe) && aligned16(rope_table),
+                "cache, c_kv, k_pe and rope_table must be 16-byte aligned");
+  MLA_CHECK_ARG(ld_c >= MLA_D_C && ld_c % 8 == 0, "ld_c must be >= 512 and a multiple of 8");
+  MLA_CHECK_ARG(ld_k >= MLA_D_R && ld_k % 8 == 0, "ld_k must be >= 64 and a multiple of 8");
+  // the absorption's, as mla_absorb_q checks them
+  if (!heads_supported(n_h))
+    return fail(MLA_ERR_UNSUPPORTED, "n_h = %d (supported: 16..128, multiple of 16)", n_h);
+  MLA_CHECK_ARG(q_nope && q_pe && w_uk && q_full, "NULL device pointer");
+  MLA_CHECK_ARG(aligned16(q_nope) && aligned16(q_pe) && aligned16(w_uk) && aligned16(q_full),
+                "pointers must be 16-byte aligned");
+  MLA_CHECK_ARG(ld_qn >= n_h * MLA_D_NOPE && ld_qn % 8 == 0, "ld_qn too small or unaligned");
+  MLA_CHECK_ARG(ld_qp >= n_h * MLA_D_R && ld_qp % 8 == 0, "ld_qp too small or unaligned");
+  mla_status_t st = require_sm100();
+  if (st != MLA_OK) return st;
+  AppendJob app;
+  app.cache = cache;
+  app.num_pages = num_pages;
+  app.block_table = block_table;
+  app.batch = batch;
+  app.max_pages = max_pages;
+  app.seq_idx = seq_idx;
+  app.pos = tok_pos;
+  app.c_kv = c_kv;
+  app.ld_c = ld_c;
+  app.k_pe = k_pe;
+  app.ld_k = ld_k;
+  app.n_tokens = n_tokens;
+  return launch_absorb_q(q_nope, ld_qn, q_pe, ld_qp, q_pos, rope_table, max_pos, w_uk, T, n_h,
+                         q_full, status, (cudaStream_t)stream, &app);
+}
+
 size_t mla_plan_bytes(int batch, int q_len, int num_ctas) {
   if (batch < 0 || q_len < 0) return 0;
   if (resolve_ctas(&num_ctas) != MLA_OK) return 0;
@@ -494,7 +546,12 @@ mla_status_t mla_gemm_bf16(const mla_bf16_t *X, int ld_x, const mla_bf16_t *W, i
 
 size_t mla_gemm_bf16_workspace_bytes(int M, int N, int K) {
   if (M <= 0 || N <= 0 || K <= 0) return 0;
-  return ((size_t)M * N * sizeof(float) + 255) & ~(size_t)255;
+  // bf16 outputs accumulate a split in M*N floats; fp32 outputs keep one
+  // partial tile per split (the projection GEMM: A = W with N rows, B = X)
+  const size_t bf16_need = ((size_t)M * N * sizeof(float) + 255) & ~(size_t)255;
+  int sms = 0;
+  if (device_info(&sms, nullptr, nullptr) != MLA_OK) return bf16_need;
+  return std::max(bf16_need, plan_gemm(N, M, K, 1, false, true, true, false, sms).part_bytes);
 }
 
 mla_status_t mla_gemm_bf16_ws(const mla_bf16_t *X, int ld_x, const mla_bf16_t *W, int ld_w,
@@ -513,11 +570,11 @@ mla_status_t mla_gemm_bf16_ws(const mla_bf16_t *X, int ld_x, const mla_bf16_t *W
   MLA_CHECK_ARG(workspace == nullptr || aligned16(workspace), "workspace must be 16-byte aligned");
   mla_status_t st = require_sm100();
   if (st != MLA_OK) return st;
-  const bool use_ws = workspace != nullptr && !c_fp32 &&
+  const bool use_ws = workspace != nullptr &&
                       workspace_bytes >= mla_gemm_bf16_workspace_bytes(M, N, K);
   return launch_projection(X, ld_x, W, ld_w, C, ld_c, c_fp32, M, N, K,
                            use_ws ? static_cast<float *>(workspace) : nullptr,
-                           (cudaStream_t)stream);
+                           use_ws ? workspace_bytes : 0, (cudaStream_t)stream);
 }
 
 size_t mla_plan_used_bytes(const void *plan_host) {

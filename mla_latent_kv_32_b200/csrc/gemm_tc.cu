@@ -30,6 +30,7 @@
 
 #include <algorithm>
 
+#include "append.cuh"
 #include "internal.h"
 #include "sm100.cuh"
 
@@ -43,6 +44,7 @@ constexpr int kSharedStages = 4;       // ring depth when CTAs share SMs
 constexpr uint32_t kSmemLimit = 232448;  // dynamic shared memory per CTA (227 KB)
 constexpr uint32_t kAStage = 128 * 128;        // 128 rows x 64 k (bf16) = 16 KB
 constexpr uint64_t kTimeoutNs = 1000000000ull;
+constexpr int kMaxPartSplits = 8;      // fp32 split-K into partial-sum tiles: at most this many
 
 struct GemmTcArgs {
   int M, N, K;          // per batch
@@ -61,6 +63,9 @@ struct GemmTcArgs {
   uint32_t *status;
   int tile_z;           // z extent of the GEMM tiles; CTAs beyond it run the side job
   int b_shared;         // every batch z reads the same B (its tensor map has one z slice)
+  int two_m;            // a CTA covers 256 rows of A: two 128-row accumulators
+  float *part;          // fp32 output split over K: split s writes its partial tile at
+                        // ((s * batch + z) * N + n) * M + m; a second kernel sums them
   // side job (rope_q_pe == nullptr: none)
   const uint16_t *rope_q_pe;
   int rope_ld_qp;
@@ -68,6 +73,7 @@ struct GemmTcArgs {
   const float *rope_table;
   int rope_max_pos, rope_T, rope_n_h;
   uint16_t *rope_q_full;
+  AppendJob app;        // second side job (n_tokens == 0: none)
 };
 
 // Side job: each thread rotates the 4 pairs of one 16-byte chunk of q^R
@@ -156,7 +162,15 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__
     // side-job CTAs: no shared memory, barriers or tensor memory
     const int per_z = gridDim.x * gridDim.y;
     const int cta = ((int)blockIdx.z - g.tile_z) * per_z + blockIdx.y * gridDim.x + blockIdx.x;
-    rope_side_job(g, cta, ((int)gridDim.z - g.tile_z) * per_z);
+    const int ctas = ((int)gridDim.z - g.tile_z) * per_z;
+    if (g.rope_q_pe != nullptr) rope_side_job(g, cta, ctas);
+    // the step's cache append: one warp per token
+    const int warps = ctas * (blockDim.x >> 5);
+    for (int t = cta * (blockDim.x >> 5) + (threadIdx.x >> 5); t < g.app.n_tokens; t += warps)
+      append_token_warp(g.app.cache, g.app.num_pages, g.app.block_table, g.app.batch,
+                        g.app.max_pages, g.app.seq_idx, g.app.pos, g.app.c_kv, g.app.ld_c,
+                        g.app.k_pe, g.app.ld_k, g.rope_table, g.rope_max_pos, t, threadIdx.x & 31,
+                        g.status);
     return;
   }
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -165,7 +179,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__
   unsigned char *smem = smem_raw + (base - raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n0 = blockIdx.x * g.BN;
-  const int m0 = blockIdx.y * 128;
+  const int m0 = blockIdx.y * (g.two_m ? 256 : 128);
+  const uint32_t a_bytes = g.two_m ? 2 * kAStage : kAStage;
   const int z = blockIdx.z / g.splits;
   const int split = blockIdx.z % g.splits;
   const int kc0 = split * g.k_chunks;
@@ -197,8 +212,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__
       const int s = i % stages;
       if (i >= stages && !wait_bar_g(bar_empty + 8 * s, ((i / stages) - 1) & 1, g.status))
         break;
-      const uint32_t a_s = base + s * g.stage_bytes, b_s = a_s + kAStage;
-      mbar_arrive_expect_tx(bar_full + 8 * s, kAStage + b_bytes);
+      const uint32_t a_s = base + s * g.stage_bytes, b_s = a_s + a_bytes;
+      mbar_arrive_expect_tx(bar_full + 8 * s, a_bytes + b_bytes);
       ++armed[s];
       if (g.a_mn) {
         // two 64-row (m) boxes of 64 k-rows each
@@ -206,6 +221,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__
         tma_load_3d(a_s + 8192, &tm_a, m0 + 64, kc * 64, z, bar_full + 8 * s);
       } else {
         tma_load_3d(a_s, &tm_a, kc * 64, m0, z, bar_full + 8 * s);
+        if (g.two_m) tma_load_3d(a_s + kAStage, &tm_a, kc * 64, m0 + 128, z, bar_full + 8 * s);
       }
       tma_load_3d(b_s, &tm_b, kc * 64, n0, g.b_shared ? 0 : z, bar_full + 8 * s);
     }
@@ -217,13 +233,16 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__
       const int s = i % stages;
       if (!wait_bar_g(bar_full + 8 * s, (i / stages) & 1, g.status)) break;
       tc_fence_after();
-      const uint32_t a_s = base + s * g.stage_bytes, b_s = a_s + kAStage;
+      const uint32_t a_s = base + s * g.stage_bytes, b_s = a_s + a_bytes;
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {
         const uint64_t ad = g.a_mn ? smem_desc(a_s + kk * 2048, 8192, 1024, kSwizzle128B)
                                    : smem_desc(a_s + kk * 32, 16, 1024, kSwizzle128B);
         const uint64_t bd = smem_desc(b_s + kk * 32, 16, 1024, kSwizzle128B);
         mma_f16_ss(tmem, ad, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+        if (g.two_m)
+          mma_f16_ss(tmem + g.BN, smem_desc(a_s + kAStage + kk * 32, 16, 1024, kSwizzle128B), bd,
+                     idesc, (i > 0 || kk > 0) ? 1u : 0u);
       }
       mma_commit(bar_empty + 8 * s);
     }
@@ -233,11 +252,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__
   // epilogue: thread = row m of the tile
   const bool done = wait_bar_g(bar_done, 0, g.status);
   tc_fence_after();
-  const int m = m0 + threadIdx.x;
   const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  for (int pass = 0; pass <= g.two_m; ++pass)
   for (int ch = 0; ch * 32 < g.BN; ++ch) {
+    const int m = m0 + 128 * pass + threadIdx.x;
     uint32_t r[32];
-    tmem_ld32(tmem + lane_off + 32 * ch, r);
+    tmem_ld32(tmem + lane_off + pass * g.BN + 32 * ch, r);
     tmem_wait_ld();
     if (!done || kc1 <= kc0 || m >= g.M) continue;
 #pragma unroll
@@ -245,6 +265,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__
       const int n = n0 + 32 * ch + e;
       if (n >= g.N) break;
       const float v = __uint_as_float(r[e]);
+      if (g.part != nullptr) {
+        g.part[(((long long)split * g.batch + z) * g.N + n) * g.M + m] = v;
+        continue;
+      }
       if (g.ws != nullptr) {
         atomicAdd(g.ws + ((long long)z * g.N + n) * g.M + m, v);
         continue;
@@ -283,6 +307,23 @@ split_to_bf16_kernel(const float *__restrict__ ws, int M, int N, int batch, uint
   }
 }
 
+// C[z][m][n] (float32, strided) = the sum over the splits of
+// part[((s * batch + z) * N + n) * M + m].
+__global__ void __launch_bounds__(256)
+part_reduce_kernel(const float *__restrict__ part, int splits, int M, int N, int batch, float *C,
+                   long long sCz, long long sCm, long long sCn) {
+  const long long total = (long long)M * N * batch;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    float acc = 0.f;
+    for (int sp = 0; sp < splits; ++sp) acc += __ldg(part + sp * total + i);
+    const int m = (int)(i % M);
+    const long long zn = i / M;
+    const int n = (int)(zn % N), z = (int)(zn / N);
+    C[(long long)z * sCz + (long long)m * sCm + (long long)n * sCn] = acc;
+  }
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   if (fn == nullptr) {
@@ -317,6 +358,49 @@ mla_status_t make_map3(CUtensorMap *tm, const void *ptr, uint64_t d0, uint64_t d
 
 }  // namespace
 
+GemmPlan plan_gemm(int M, int N, int K, int batch, bool a_mn, bool c_fp32, bool fp32_part,
+                   bool atomic_split, int sms) {
+  GemmPlan pl;
+  pl.BN = N >= 256 ? 256 : ((N + 15) / 16) * 16;
+  pl.ntile = (N + pl.BN - 1) / pl.BN;
+  const int kchunks = (K + 63) / 64;
+  const bool big_m = !a_mn && M >= 1024;
+  pl.splits = 1;
+  pl.part = false;
+  if (c_fp32 && fp32_part) {
+    // fp32 output with a workspace: 256-row tiles (two accumulators, so each
+    // CTA reads the B tile for twice the rows), split over K into partial-sum
+    // tiles until the grid fills one wave (at most kMaxPartSplits; W^O at 256
+    // tokens: 113.7 -> 95 us)
+    pl.two_m = big_m;
+    pl.mtile = (M + (pl.two_m ? 255 : 127)) / (pl.two_m ? 256 : 128);
+    const long long tiles = (long long)pl.ntile * pl.mtile * batch;
+    if (tiles < sms) {
+      const int s0 = (int)std::min<long long>(std::min<long long>(sms / tiles, kMaxPartSplits),
+                                              kchunks / 2);
+      if (s0 >= 2) {
+        const int per = (kchunks + s0 - 1) / s0;
+        pl.splits = (kchunks + per - 1) / per;   // no empty split
+        pl.part = pl.splits > 1;
+      }
+    }
+  } else {
+    // otherwise a small tile grid splits over K with atomic adds on 128-row
+    // tiles (the fp32 output, or a bf16 output's fp32 workspace); a grid that
+    // does not split takes 256-row tiles
+    const long long tiles1 = (long long)pl.ntile * ((M + 127) / 128) * batch;
+    if (atomic_split)
+      while (pl.splits < 32 && tiles1 * pl.splits * 2 <= 296 && kchunks / (pl.splits * 2) >= 4)
+        pl.splits *= 2;
+    pl.two_m = big_m && pl.splits == 1;
+    pl.mtile = (M + (pl.two_m ? 255 : 127)) / (pl.two_m ? 256 : 128);
+  }
+  pl.k_chunks = (kchunks + pl.splits - 1) / pl.splits;
+  pl.part_bytes =
+      pl.part ? ((size_t)pl.splits * M * N * batch * sizeof(float) + 255) & ~(size_t)255 : 0;
+  return pl;
+}
+
 mla_status_t launch_gemm_tc(const GemmTcDesc &d, cudaStream_t stream) {
   if (d.M == 0 || d.N == 0 || d.batch == 0) return MLA_OK;
   if (d.K <= 0 || d.K % 16 != 0) return fail(MLA_ERR_UNSUPPORTED, "GEMM K must be a multiple of 16");
@@ -337,32 +421,37 @@ mla_status_t launch_gemm_tc(const GemmTcDesc &d, cudaStream_t stream) {
   g.N = d.N;
   g.K = d.K;
   g.BN = BN;
+  int sms = 0;
+  st = device_info(&sms, nullptr, nullptr);
+  if (st != MLA_OK) return st;
+  const GemmPlan pl = plan_gemm(d.M, d.N, d.K, d.batch, d.a_mn, d.c_fp32 != 0,
+                                d.c_fp32 && d.part_ws != nullptr,
+                                (d.c_fp32 && d.allow_split) || (!d.c_fp32 && d.split_ws != nullptr),
+                                sms);
+  if (pl.part && d.part_ws_bytes < pl.part_bytes)
+    return fail(MLA_ERR_WORKSPACE_TOO_SMALL, "GEMM workspace %zu B < %zu B", d.part_ws_bytes,
+                pl.part_bytes);
   const int kchunks = (d.K + 63) / 64;
-  const int ntile = (d.N + BN - 1) / BN, mtile = (d.M + 127) / 128;
-  int splits = 1;
-  if ((d.c_fp32 && d.allow_split) || (!d.c_fp32 && d.split_ws != nullptr)) {
-    // spread long reductions over more CTAs when the tile grid is small
-    const int ctas = ntile * mtile * d.batch;
-    while (splits < 32 && ctas * splits * 2 <= 296 && kchunks / (splits * 2) >= 4) splits *= 2;
-  }
+  const bool two_m = pl.two_m;
+  const int ntile = pl.ntile, mtile = pl.mtile;
+  const int splits = pl.splits;
   const bool ws_split = splits > 1 && !d.c_fp32;
+  g.part = pl.part ? d.part_ws : nullptr;
   g.splits = splits;
   g.k_chunks = (kchunks + splits - 1) / splits;
-  g.stage_bytes = kAStage + (((uint32_t)BN * 128 + 1023u) & ~1023u);
+  g.stage_bytes = (two_m ? 2 : 1) * kAStage + (((uint32_t)BN * 128 + 1023u) & ~1023u);
+  g.two_m = two_m ? 1 : 0;
   // A grid that fits one CTA per SM keeps every k-chunk of a tile in flight
   // (up to kMaxStages, within the shared memory), so a tile waits one load
   // round trip rather than one per ring cycle; denser grids keep a shallower
   // ring and several CTAs per SM.
-  int sms = 0;
-  st = device_info(&sms, nullptr, nullptr);
-  if (st != MLA_OK) return st;
   const uint32_t bar_bytes = 8 * (2 * kMaxStages + 2);
   const int fit = (int)((kSmemLimit - 1024 - bar_bytes) / g.stage_bytes);
   const long long tile_ctas = (long long)ntile * mtile * d.batch * splits;
-  const int depth = tile_ctas <= sms ? std::min(kMaxStages, fit) : kSharedStages;
+  const int depth = tile_ctas <= sms ? std::min(kMaxStages, fit) : std::min(kSharedStages, fit);
   g.stages = std::min(g.k_chunks, depth);
   g.tmem_cols = 32;
-  while (g.tmem_cols < (uint32_t)BN) g.tmem_cols *= 2;
+  while (g.tmem_cols < (uint32_t)(two_m ? 2 * BN : BN)) g.tmem_cols *= 2;
   const uint32_t smem_bytes = g.stages * g.stage_bytes + bar_bytes + 1024;
   g.batch = d.batch;
   g.a_mn = d.a_mn;
@@ -383,17 +472,18 @@ mla_status_t launch_gemm_tc(const GemmTcDesc &d, cudaStream_t stream) {
   g.rope_T = d.rope_T;
   g.rope_n_h = d.rope_n_h;
   g.rope_q_full = d.rope_q_full;
+  g.app = d.app;
   // side-job CTAs: whole z-slices of the grid, ~64 CTAs of 128 threads
   int side_z = 0;
-  if (d.rope_q_pe != nullptr && d.rope_T > 0) {
-    const long long chunks = (long long)d.rope_T * d.rope_n_h * 8;
-    const long long want = std::min<long long>(64, (chunks + 127) / 128);
-    side_z = (int)((want + ntile * mtile - 1) / (ntile * mtile));
-  }
+  long long want = 0;
+  if (d.rope_q_pe != nullptr && d.rope_T > 0)
+    want = std::min<long long>(64, ((long long)d.rope_T * d.rope_n_h * 8 + 127) / 128);
+  if (d.app.n_tokens > 0) want = std::max<long long>(want, std::min(64, (d.app.n_tokens + 3) / 4));
+  if (want > 0) side_z = (int)((want + ntile * mtile - 1) / (ntile * mtile));
   if (ws_split) {
     MLA_CUDA_TRY(cudaMemsetAsync(d.split_ws, 0, (size_t)d.M * d.N * d.batch * sizeof(float),
                                  stream));
-  } else if (splits > 1) {
+  } else if (splits > 1 && !pl.part) {
     if (!d.c_contiguous)
       return fail(MLA_ERR_UNSUPPORTED, "split-K needs a contiguous fp32 output");
     MLA_CUDA_TRY(cudaMemsetAsync(d.C, 0, d.c_bytes, stream));
@@ -403,6 +493,14 @@ mla_status_t launch_gemm_tc(const GemmTcDesc &d, cudaStream_t stream) {
   dim3 grid(ntile, mtile, d.batch * splits + side_z);
   gemm_tc_kernel<<<grid, 128, smem_bytes, stream>>>(tm_a, tm_b, g);
   MLA_LAUNCH_CHECK("gemm_tc_kernel");
+  if (pl.part) {
+    const long long total = (long long)d.M * d.N * d.batch;
+    const int blocks = (int)std::min<long long>(4 * sms, (total + 255) / 256);
+    part_reduce_kernel<<<blocks, 256, 0, stream>>>(d.part_ws, splits, d.M, d.N, d.batch,
+                                                    static_cast<float *>(d.C), d.sCz, d.sCm,
+                                                    d.sCn);
+    MLA_LAUNCH_CHECK("part_reduce_kernel");
+  }
   if (ws_split) {
     const long long total = (long long)d.M * d.N * d.batch;
     const int blocks = (int)std::min<long long>(1184, (total + 255) / 256);

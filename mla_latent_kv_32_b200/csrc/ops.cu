@@ -9,7 +9,7 @@ namespace mla {
 mla_status_t launch_absorb_q(const uint16_t *q_nope, int ld_qn, const uint16_t *q_pe, int ld_qp,
                              const int32_t *pos, const float *rope_table, int max_pos,
                              const uint16_t *w_uk, int T, int n_h, uint16_t *q_full,
-                             uint32_t *status, cudaStream_t stream) {
+                             uint32_t *status, cudaStream_t stream, const AppendJob *app) {
   GemmTcDesc d = {};
   d.A = w_uk; d.sAz = (long long)MLA_D_NOPE * MLA_D_C; d.sAk = MLA_D_C; d.a_mn = 1;
   d.B = q_nope; d.sBz = MLA_D_NOPE; d.sBn = ld_qn;
@@ -18,6 +18,7 @@ mla_status_t launch_absorb_q(const uint16_t *q_nope, int ld_qn, const uint16_t *
   d.status = status;
   d.rope_q_pe = q_pe; d.rope_ld_qp = ld_qp; d.rope_pos = pos; d.rope_table = rope_table;
   d.rope_max_pos = max_pos; d.rope_T = T; d.rope_n_h = n_h; d.rope_q_full = q_full;
+  if (app != nullptr) d.app = *app;
   return launch_gemm_tc(d, stream);
 }
 
@@ -35,8 +36,8 @@ mla_status_t launch_out_absorb(const uint16_t *o_latent, const uint16_t *w_uv, i
 
 // C[t][f] = sum_k X[t][k] * W[f][k]   (m = output feature f, n = token t)
 mla_status_t launch_projection(const uint16_t *X, int ld_x, const uint16_t *W, int ld_w, void *C,
-                               int ld_c, int c_fp32, int M, int N, int K, float *split_ws,
-                               cudaStream_t stream) {
+                               int ld_c, int c_fp32, int M, int N, int K, float *ws,
+                               size_t ws_bytes, cudaStream_t stream) {
   GemmTcDesc d = {};
   d.A = W; d.sAz = 0; d.sAm = ld_w; d.a_mn = 0;
   d.B = X; d.sBz = 0; d.sBn = ld_x;
@@ -45,7 +46,9 @@ mla_status_t launch_projection(const uint16_t *X, int ld_x, const uint16_t *W, i
   d.allow_split = c_fp32;
   d.c_contiguous = 1;
   d.c_bytes = (size_t)M * ld_c * (c_fp32 ? 4 : 2);
-  d.split_ws = c_fp32 ? nullptr : split_ws;
+  d.split_ws = c_fp32 ? nullptr : ws;
+  d.part_ws = c_fp32 ? ws : nullptr;
+  d.part_ws_bytes = c_fp32 ? ws_bytes : 0;
   return launch_gemm_tc(d, stream);
 }
 

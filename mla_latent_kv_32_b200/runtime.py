@@ -172,9 +172,20 @@ class DecodeSession(_GraphStep):
     def expand(self, stream=None):
         mla.mla_out_absorb(self.o, self.w_uv, self.T, self.n_h, self.u, self.n_h * D_V, stream)
 
+    def append_absorb(self, stream=None):
+        """append + absorb in one launch (the bf16 cache)."""
+        mla.mla_append_absorb_q(self.cache, self.num_pages, self.table, self.B, self.max_pages,
+                                self.seq_idx, self.pos, self.c_new, D_C, self.k_new, D_R, self.T,
+                                self.q_nope, self.n_h * D_NOPE, self.q_pe, self.n_h * D_R,
+                                self.w_uk, self.pos, self.rope, self.max_pos, self.T, self.n_h,
+                                self.q_full, self.status, stream)
+
     def step(self, stream=None):
-        self.append(stream)
-        self.absorb(stream)
+        if self.fp8:
+            self.append(stream)
+            self.absorb(stream)
+        else:
+            self.append_absorb(stream)
         self.attend(stream)
         self.expand(stream)
 
@@ -322,31 +333,38 @@ class LayerSession(_GraphStep):
 
     # the layer's calls one by one (step runs them in this order) -------------
     def _gemm_ws(self):
-        # split-K workspace of the two down-projections from the hidden state
+        # split-K partial-sum workspace shared by the layer's projections (the
+        # calls run one after another on one stream)
         if getattr(self, "gemm_ws", None) is None:
-            need = max(mla.mla_gemm_bf16_workspace_bytes(self.Tq, max(self.q_lora, 1), self.hidden),
-                       mla.mla_gemm_bf16_workspace_bytes(self.T, ROW, self.hidden))
+            n_h, d, Tq = self.n_h, self.hidden, self.Tq
+            q_in = self.q_lora or d
+            shapes = [(Tq, n_h * (D_NOPE + D_R), q_in), (self.T, ROW, d), (Tq, d, n_h * D_V),
+                      (Tq, n_h * D_R, q_in), (Tq, d, n_h * D_C)]
+            if self.q_lora:
+                shapes.append((Tq, self.q_lora, d))
+            need = max(mla.mla_gemm_bf16_workspace_bytes(*sh) for sh in shapes)
             self.gemm_ws = torch.empty(max(need, 256), dtype=torch.uint8, device=self.device)
         return self.gemm_ws
+
+    def _gemm(self, X, ld_x, W, ld_w, C, ld_c, c_fp32, M, N, K, stream):
+        ws = self._gemm_ws()
+        mla.mla_gemm_bf16_ws(X, ld_x, W, ld_w, C, ld_c, c_fp32, M, N, K, ws, ws.numel(), stream)
 
     def project_q(self, stream=None):
         n_h, d = self.n_h, self.hidden
         hq = self.h[self.T - self.Tq:]
         nq = n_h * (D_NOPE + D_R)
         if self.q_lora:
-            ws = self._gemm_ws()
-            mla.mla_gemm_bf16_ws(hq, d, self.w_dq, d, self.cq, self.q_lora, 0, self.Tq,
-                                 self.q_lora, d, ws, ws.numel(), stream)
-            mla.mla_gemm_bf16(self.cq, self.q_lora, self.w_qcat, self.q_lora, self.q, nq, 0,
-                              self.Tq, nq, self.q_lora, stream)
+            self._gemm(hq, d, self.w_dq, d, self.cq, self.q_lora, 0, self.Tq, self.q_lora, d,
+                       stream)
+            self._gemm(self.cq, self.q_lora, self.w_qcat, self.q_lora, self.q, nq, 0, self.Tq, nq,
+                       self.q_lora, stream)
         else:
-            mla.mla_gemm_bf16(hq, d, self.w_qcat, d, self.q, nq, 0, self.Tq, nq, d, stream)
+            self._gemm(hq, d, self.w_qcat, d, self.q, nq, 0, self.Tq, nq, d, stream)
 
     def project_kv(self, stream=None):
         d = self.hidden
-        ws = self._gemm_ws()
-        mla.mla_gemm_bf16_ws(self.h, d, self.w_kvcat, d, self.kv, ROW, 0, self.T, ROW, d, ws,
-                             ws.numel(), stream)
+        self._gemm(self.h, d, self.w_kvcat, d, self.kv, ROW, 0, self.T, ROW, d, stream)
 
     def append(self, stream=None):
         kv_pe = self.kv[:, D_C:]
@@ -361,6 +379,17 @@ class LayerSession(_GraphStep):
         mla.mla_absorb_q(self.q, nq, q_pe, nq, self.w_uk, self.q_pos, self.rope, self.max_pos,
                          self.Tq, n_h, self.q_full, self.status, stream)
 
+    def append_absorb(self, stream=None):
+        """append (every token entering the layer) + absorb (the query tokens)
+        in one launch."""
+        n_h = self.n_h
+        nq = n_h * (D_NOPE + D_R)
+        mla.mla_append_absorb_q(self.cache, self.num_pages, self.table, self.B, self.max_pages,
+                                self.tok_seq, self.tok_pos, self.kv, ROW, self.kv[:, D_C:], ROW,
+                                self.T, self.q, nq, self.q[:, n_h * D_NOPE:], nq, self.w_uk,
+                                self.q_pos, self.rope, self.max_pos, self.Tq, n_h, self.q_full,
+                                self.status, stream)
+
     def attend(self, stream=None):
         mla.mla_decode_attention(self.q_full, self.cache, self.num_pages, self.table,
                                  self.max_pages, self.B, self.q_len, self.n_h, self.scale,
@@ -373,22 +402,20 @@ class LayerSession(_GraphStep):
 
     def project_out(self, stream=None):
         n_h, d = self.n_h, self.hidden
-        mla.mla_gemm_bf16(self.u, n_h * D_V, self.w_o, n_h * D_V, self.out, d, 1, self.Tq, d,
-                          n_h * D_V, stream)
+        self._gemm(self.u, n_h * D_V, self.w_o, n_h * D_V, self.out, d, 1, self.Tq, d, n_h * D_V,
+                   stream)
 
     # the folded step's own calls ---------------------------------------------
     def project_q_folded(self, stream=None):
         n_h, d = self.n_h, self.hidden
         hq = self.h[self.T - self.Tq:]
         if self.q_lora:
-            ws = self._gemm_ws()
-            mla.mla_gemm_bf16_ws(hq, d, self.w_dq, d, self.cq, self.q_lora, 0, self.Tq,
-                                 self.q_lora, d, ws, ws.numel(), stream)
+            self._gemm(hq, d, self.w_dq, d, self.cq, self.q_lora, 0, self.Tq, self.q_lora, d,
+                       stream)
             x, ld = self.cq, self.q_lora
         else:
             x, ld = hq, d
-        mla.mla_gemm_bf16(x, ld, self.w_qr, ld, self.q_r, n_h * D_R, 0, self.Tq, n_h * D_R, ld,
-                          stream)
+        self._gemm(x, ld, self.w_qr, ld, self.q_r, n_h * D_R, 0, self.Tq, n_h * D_R, ld, stream)
 
     def absorb_folded(self, stream=None):
         n_h = self.n_h
@@ -399,8 +426,8 @@ class LayerSession(_GraphStep):
 
     def project_out_folded(self, stream=None):
         n_h, d = self.n_h, self.hidden
-        mla.mla_gemm_bf16(self.o, n_h * D_C, self.w_o_f, n_h * D_C, self.out, d, 1, self.Tq, d,
-                          n_h * D_C, stream)
+        self._gemm(self.o, n_h * D_C, self.w_o_f, n_h * D_C, self.out, d, 1, self.Tq, d, n_h * D_C,
+                   stream)
 
     def step(self, stream=None):
         if self.folded:
@@ -413,8 +440,7 @@ class LayerSession(_GraphStep):
             return
         self.project_q(stream)
         self.project_kv(stream)
-        self.append(stream)
-        self.absorb(stream)
+        self.append_absorb(stream)
         self.attend(stream)
         self.expand(stream)
         self.project_out(stream)

@@ -63,23 +63,30 @@ def test_layer(dev, name):
     assert np.array_equal(got_all, want), "appended cache rows are not bit-exact"
 
 
-@pytest.mark.parametrize("M,N,K", [(256, 576, 7168), (256, 1536, 7168), (7, 64, 512)])
-def test_split_k_gemm_matches_fp32(dev, M, N, K):
-    # C = X W^T with a workspace (split over K for the long reductions) against
-    # a float64 product of the same bf16 inputs; bf16 output
+@pytest.mark.parametrize("M,N,K,fp32", [
+    (256, 576, 7168, 0), (256, 1536, 7168, 0), (7, 64, 512, 0), (256, 24576, 1536, 0),
+    (256, 7168, 16384, 1), (100, 1100, 640, 1), (3, 2048, 1024, 0)])
+def test_split_k_gemm_matches_fp32(dev, M, N, K, fp32):
+    # C = X W^T with a workspace (split over K into partial sums when the tile
+    # grid is below one wave; 256-row weight tiles from 1024 rows up) and
+    # without one (fp32 outputs may split with atomic adds), against a float64
+    # product of the same bf16 inputs
     g = torch.Generator().manual_seed(M * 7 + N)
     X = (torch.randn(M, K, generator=g) / math.sqrt(K)).to(torch.bfloat16)
     W = torch.randn(N, K, generator=g).to(torch.bfloat16)
     ref = (X.double() @ W.double().T).numpy()
     Xd, Wd = X.to(dev), W.to(dev)
-    C = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
-    ws = torch.empty(mla.mla_gemm_bf16_workspace_bytes(M, N, K), dtype=torch.uint8, device=dev)
-    mla.mla_gemm_bf16_ws(Xd, K, Wd, K, C, N, 0, M, N, K, ws, ws.numel())
+    dt = torch.float32 if fp32 else torch.bfloat16
+    C = torch.full((M, N), float("nan"), dtype=dt, device=dev)
+    need = mla.mla_gemm_bf16_workspace_bytes(M, N, K)
+    ws = torch.full((max(need, 256),), 0xFF, dtype=torch.uint8, device=dev)   # NaN-poisoned
+    mla.mla_gemm_bf16_ws(Xd, K, Wd, K, C, N, fp32, M, N, K, ws, ws.numel())
     got = C.float().cpu().numpy()
-    C2 = torch.empty_like(C)
-    mla.mla_gemm_bf16(Xd, K, Wd, K, C2, N, 0, M, N, K)
+    C2 = torch.full_like(C, float("nan"))
+    mla.mla_gemm_bf16(Xd, K, Wd, K, C2, N, fp32, M, N, K)
     got2 = C2.float().cpu().numpy()
     for g_ in (got, got2):
+        assert np.all(np.isfinite(g_))
         err = np.abs(g_ - ref)
         assert err.max() <= 2e-2 * np.abs(ref).max() and err.sum() <= 5e-3 * np.abs(ref).sum()
 
