@@ -39,6 +39,10 @@ METRIC = "MLA decode tokens/sec and cache GB/s (% of HBM/bf16 roofline) on 1 B20
 UNIT = "tokens/s"
 ROW_BYTES = 1152                 # 576 bf16 per cached token
 FP8_TOKEN_BYTES = 644            # FP8 cache: 512 E4M3 + 64 bf16 + a float32 scale
+# independent batches in flight in the end-to-end loop: with two, each
+# stream's upload -> step -> download chain (~0.26 ms on v3) paced the loop
+# at 0.23 ms per step; with three the step's compute does (0.14 ms)
+E2E_SESSIONS = 3
 FLOP_PER_TOKEN_HEAD = 2 * 576 + 2 * 512
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # B200 data-sheet figures (dense bf16), reported beside the measured peaks
@@ -53,10 +57,14 @@ def dist_stats(xs):
 
 # DRAM traffic per launch of mla_decode_attention measured by ncu
 # (dram__bytes_read.sum + dram__bytes_write.sum), keyed by the SHA-256 of the
-# decode sources it was measured on and the workload; reported only while the
-# sources match (the combine kernel's few MB are not included).
+# decode sources it was measured on, the workload and the cache format;
+# reported only while the sources match (the combine kernel's few MB are not
+# included).
 TRAFFIC = {
-    ("79c6a9d1edad444d", "v3"): 317488384,   # decode_pair_kernel<bf16>, 1.051 x the cache bytes
+    # decode_pair_kernel<bf16>: 1.054 x the cache bytes
+    ("d754049324a228ee", "v3", "bf16"): 318256128,
+    # decode_pair_kernel<fp8>: 1.066 x the cache bytes read, 8.6 MB written
+    ("d754049324a228ee", "v3", "fp8"): 188447232,
 }
 
 
@@ -692,22 +700,25 @@ def main():
             cache_bytes = int(inp.lens.sum()) * FP8_TOKEN_BYTES
 
         # e2e: per-step inputs uploaded from pinned host memory and the result
-        # read back to pinned host memory, through the library's calls. Two
+        # read back to pinned host memory, through the library's calls. Three
         # independent sessions (each with its own cache, weights and I/O
-        # buffers) each hold one CUDA graph of upload + four calls + download
-        # and alternate steps on two streams, so one batch's copies overlap
-        # the other's compute. Every step touches more than L2 holds, so no
-        # flush runs in this loop.
+        # buffers) each hold one CUDA graph of upload + the step's calls +
+        # download and take turns on three streams, so one batch's copies
+        # overlap the others' compute, and one batch's GEMMs run on the SMs
+        # another batch's attention leaves idle. Every step touches more than
+        # L2 holds, so no flush runs in this loop.
         e2e = None
         if not args.no_e2e:
-            sess2 = DecodeSession(inp, dev, num_ctas=args.num_ctas, max_split=args.max_split,
-                                  fp8=fp8)
-            pair = [sess, sess2]
+            sessions = [sess] + [DecodeSession(inp, dev, num_ctas=args.num_ctas,
+                                               max_split=args.max_split, fp8=fp8)
+                                 for _ in range(E2E_SESSIONS - 1)]
             ins, host_in, host_out0 = sess.pinned_step_buffers()
-            host_outs = [host_out0, torch.empty_like(host_out0).pin_memory()]
+            host_outs = [host_out0] + [torch.empty_like(host_out0).pin_memory()
+                                       for _ in range(E2E_SESSIONS - 1)]
             h2d, d2h = DecodeSession.step_io_bytes(ins, host_out0)
-            graphs = [capture_io_step(s_, host_in, host_outs[i]) for i, s_ in enumerate(pair)]
-            streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+            graphs = [capture_io_step(s_, host_in, host_outs[i])
+                      for i, s_ in enumerate(sessions)]
+            streams = [torch.cuda.Stream() for _ in sessions]
             run_e2e_graphs(graphs, streams, 8)
             torch.cuda.synchronize()
             E = max(args.e2e_steps, K)
@@ -723,7 +734,7 @@ def main():
             barrier()
             t_e2e = e0.elapsed_time(e1) / E
             (t_e2e,) = max_over_ranks([t_e2e], dist, dev, world)
-            for s_ in pair:
+            for s_ in sessions:
                 assert s_.read_status() == 0, "device status in the end-to-end loop"
             # the host link alone: the same per-step copies timed by themselves
             def copy_ms(fn, n=20):
@@ -745,12 +756,13 @@ def main():
                                  "h2d_gbs": h2d / t_h2d / 1e6, "d2h_gbs": d2h / t_d2h / 1e6},
                    "ms_per_step": t_e2e, "steps": E,
                    "host_enqueue_us_per_step": host_s / E * 1e6,
-                   "method": "two sessions, each one CUDA graph of upload (pinned host -> "
-                             "device) + the four library calls + download (device -> pinned "
-                             "host); steps alternate on two streams so one batch's copies "
-                             "overlap the other's compute; no L2 flush (each step touches "
-                             "> L2)"}
-            del graphs, sess2
+                   "method": f"{E2E_SESSIONS} sessions (independent batches), each one "
+                             "CUDA graph of upload (pinned host -> device) + the step's "
+                             "library calls + download (device -> pinned host); steps take "
+                             f"turns on {E2E_SESSIONS} streams so one batch's copies and "
+                             "GEMMs overlap another's attention; no L2 flush (each step "
+                             "touches > L2)"}
+            del graphs, sessions
 
         configs = {}
         if not args.no_configs and world == 1:
@@ -771,7 +783,7 @@ def main():
     t_mem = cache_bytes / (peaks["hbm_gbs"] * 1e9)
     t_tc = flops / (peaks["bf16_tflops"] * 1e12)
     src_hash = decode_sources_hash()
-    traffic = TRAFFIC.get((src_hash, args.workload))
+    traffic = TRAFFIC.get((src_hash, args.workload, args.cache))
     roof = {
         "kernel": "mla_decode_attention (decode + combine kernels)",
         "bound": "hbm" if t_mem >= t_tc else "tensor",

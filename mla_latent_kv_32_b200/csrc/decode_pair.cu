@@ -35,6 +35,20 @@
 // row's max grows by more than 8 (log2 units); the final normalisation uses the
 // same reference max, so the result is exact up to rounding.
 //
+// FP8 cache instance (448 threads: warps 10-13 convert). The stages run in
+// the same order, each loaded to its own CTA's barriers and expanded in place
+// before the MMA issuer takes it: a score chunk pair lands as the pages' 128
+// code columns in the first of its two stages, an output stage as one page's
+// code columns in its upper half, and the converter warp that owns the stage
+// writes code * scale as fp16 over the stage (each row overwrites only its
+// own codes). The latent MMAs take fp16 operands: the query's latent columns
+// are converted to fp16 when they land (exact for the bf16 values in the
+// fp16 range), the probabilities are rounded to fp16, and code * scale is
+// exact on the fp16 grid for scales in [2^-15, 2^7]. The RoPE chunk (bf16 k^R
+// and q^R) stays bf16 with its own bf16 MMA into the same accumulator. A value
+// outside the fp16 range sets MLA_DEV_RANGE. The producer brings each tile's
+// pages into L2 one tile ahead.
+//
 // Every wait is bounded (about one second); on expiry the kernel sets
 // MLA_DEV_TIMEOUT, stops issuing work, drains what it issued and exits.
 #include <cuda.h>
@@ -55,7 +69,6 @@ constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr int kConvWarp0 = 10;                       // FP8 cache: converter warps 10..13
 constexpr int kConvWarps = 4;
-constexpr int kConvThreads = 32 * kConvWarps;
 constexpr int kTilePages = 4;                       // pages per score tile (256 tokens)
 constexpr int kChunksQK = MLA_ROW / 64;              // 9 column chunks of the score MMA
 constexpr uint32_t kBox = 64 * 128;                  // 64 rows x 64 bf16, 128-byte swizzle
@@ -63,19 +76,23 @@ constexpr uint32_t kStageBytes = 2 * kBox;           // 16384
 constexpr uint32_t kOffQ = 0;                        // 9 x [64 heads][64 cols]
 constexpr uint32_t kOffP = kOffQ + kChunksQK * kBox; // 73728: 4 x [64 heads][64 tokens]
 constexpr uint32_t kOffRing = kOffP + kTilePages * kBox;  // 106496: bf16 operand stages
-constexpr uint32_t kLandStride = kBox + 1024;        // FP8 landing slot: 8 KB rows + scales
+constexpr uint32_t kHalfStage = kStageBytes / 2;     // FP8: codes land in a stage's upper half
+constexpr uint32_t kScaleSlot = 512;                 // FP8: the scales of a stage's <= 2 pages
 constexpr uint32_t kBarArea = 384;
 
 constexpr int kMaxStages = 7;                        // capacity of the stage barrier arrays
-constexpr int kMaxLand = 9;                          // capacity of the landing barrier arrays
+// FP8: the producer brings a tile's pages into L2 this many tiles before it
+// loads them. With half the bytes of a bf16 stage in each stage, the ring
+// keeps too few bytes in flight to cover a load from HBM.
+constexpr int kFp8PrefetchTiles = 1;
 
 enum {
   B_FULL0 = 0,                          // [kMaxStages] stage ready (even CTA)
   B_EMPTY0 = B_FULL0 + kMaxStages,      // [kMaxStages] stage consumed (both CTAs)
-  B_LFULL0 = B_EMPTY0 + kMaxStages,     // [kMaxLand] FP8 landing slot loaded (local)
-  B_LEMPTY0 = B_LFULL0 + kMaxLand,      // [kMaxLand] FP8 landing slot converted (local)
-  B_QFULL = B_LEMPTY0 + kMaxLand,       // query rows loaded (even CTA: both CTAs' bytes)
+  B_LFULL0 = B_EMPTY0 + kMaxStages,     // [kMaxStages] FP8 codes of a stage landed (local)
+  B_QFULL = B_LFULL0 + kMaxStages,      // query rows loaded (even CTA: both CTAs' bytes)
   B_QEMPTY,                        // last score MMA of the item done (both)
+  B_QCONV,                         // FP8: query rows converted to fp16 (even CTA: 8 warps)
   B_SFULL0, B_SFULL1,              // scores of a tile ready (both)
   B_SFREE0, B_SFREE1,              // scores read out (even CTA: 16 warps of both CTAs)
   B_PFULL,                         // P written (even CTA: 16 warps)
@@ -87,25 +104,24 @@ enum {
 };
 static_assert(8 * B_COUNT + 8 <= kBarArea, "barrier area overflow");
 
-// Shared-memory layout of the two instances. bf16 cache: a 7-stage ring of
-// bf16 operand stages filled by TMA. FP8 cache: a 4-stage ring of the same
-// bf16 stages, written by converter warps from a 6-slot ring of FP8 landing
-// slots (one page x 128 byte columns, plus the page's 64 token scales).
+// Shared-memory layout of the two instances: a 7-stage ring of bf16 operand
+// stages. bf16 cache: TMA fills the stages. FP8 cache: TMA lands a stage's
+// E4M3 codes in its upper half (and the tokens' scales in the stage's scale
+// slot), and the converter warps expand them in place into the bf16 stage.
 template <bool kFp8>
 struct Cfg {
   static constexpr int kThreads = kFp8 ? 32 * (kConvWarp0 + kConvWarps) : 320;
-  static constexpr int kStages = kFp8 ? 2 : 7;
-  static constexpr int kLand = kFp8 ? 9 : 0;
-  static constexpr uint32_t kOffLand = kOffRing + kStages * kStageBytes;
-  static constexpr uint32_t kOffBar = kOffLand + kLand * kLandStride;
+  static constexpr int kStages = 7;
+  static constexpr uint32_t kOffScale = kOffRing + kStages * kStageBytes;
+  static constexpr uint32_t kOffBar = kOffScale + (kFp8 ? kStages * kScaleSlot : 0);
   static constexpr uint32_t kOffTmemPtr = kOffBar + 8 * B_COUNT;
   static constexpr uint32_t kOffAbort = kOffTmemPtr + 4;
   static constexpr uint32_t kOffPM = kOffBar + kBarArea;  // row maxes [2 parity][4 pages][64]
   static constexpr uint32_t kOffPL = kOffPM + 2 * 4 * 64 * 4;  // row sums [4 pages][64]
   static constexpr uint32_t kSmemBytes = kOffPL + 4 * 64 * 4;
   static_assert(kSmemBytes <= 232448, "shared memory budget");
-  static_assert((kOffLand & 1023) == 0 && (kLandStride & 1023) == 0, "landing alignment");
-  static_assert(kStages <= kMaxStages && kLand <= kMaxLand, "barrier arrays too small");
+  static_assert((kOffScale & 15) == 0, "scale slot alignment");
+  static_assert(kStages <= kMaxStages, "barrier arrays too small");
 };
 
 constexpr uint32_t kTmemCols = 512;
@@ -126,6 +142,7 @@ struct PairArgs {
   uint64_t wait_ns;     // bound of every barrier wait
   int suppress_arrive;  // test hook: skip the first arrival on stage 0
   const float *scales;  // FP8 cache: [num_pages][64] per-token scales
+  const unsigned char *fp8_pool;  // FP8 cache: [num_pages][64][640] (L2 prefetch)
 };
 
 struct Ctx {
@@ -207,32 +224,36 @@ __device__ __forceinline__ uint32_t pack_hi_pair(uint32_t a_hi, uint32_t b_hi) {
 
 __device__ __forceinline__ int tiles_of(int np) { return (np + kTilePages - 1) / kTilePages; }
 
-// E4M3 -> float by bit placement: the code's sign goes to bit 31 and its 7
-// exponent/mantissa bits to bits 26..20, which is the float 2^-120 times the
-// code's value for normal and subnormal codes alike (the E4M3 subnormal
-// 0.mmm x 2^-6 lands on the float subnormal 0.mmm x 2^-126). Multiplying by
-// 2^120 and then by the power-of-two scale is exact, and so is keeping the
-// upper 16 bits as the bf16 value (4 significant bits). Integer and FMA
-// pipes only.
-// 16 E4M3 codes (16 bytes, element 0 lowest) -> 16 bf16 values code * sc.
-__device__ __forceinline__ void fp8x16_to_bf16(const uint4 &v, float sc, uint4 &o0, uint4 &o1) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-  const float k120 = 1.329227995784916e36f;   // 2^120
-  uint32_t r[8];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const uint32_t x = w[i];
-    const uint32_t f0 = ((x << 24) & 0x80000000u) | ((x << 20) & 0x07F00000u);
-    const uint32_t f1 = ((x << 16) & 0x80000000u) | ((x << 12) & 0x07F00000u);
-    const uint32_t f2 = ((x << 8) & 0x80000000u) | ((x << 4) & 0x07F00000u);
-    const uint32_t f3 = (x & 0x80000000u) | ((x >> 4) & 0x07F00000u);
-    const float g0 = __uint_as_float(f0) * k120 * sc, g1 = __uint_as_float(f1) * k120 * sc;
-    const float g2 = __uint_as_float(f2) * k120 * sc, g3 = __uint_as_float(f3) * k120 * sc;
-    r[2 * i] = __byte_perm(__float_as_uint(g0), __float_as_uint(g1), 0x7632);
-    r[2 * i + 1] = __byte_perm(__float_as_uint(g2), __float_as_uint(g3), 0x7632);
-  }
-  o0 = make_uint4(r[0], r[1], r[2], r[3]);
-  o1 = make_uint4(r[4], r[5], r[6], r[7]);
+// fp16 helpers of the FP8 instance (its MMA operands are fp16: every E4M3
+// code times a power-of-two scale, every bf16 query and k^R value in the
+// normal fp16 range, and the probabilities are exact or correctly rounded
+// there).
+// 4 E4M3 codes (element 0 lowest) -> two packed fp16 pairs, exactly.
+__device__ __forceinline__ void e4m3x4_to_f16x2(uint32_t w, uint32_t &d0, uint32_t &d1) {
+  asm("{\n .reg .b16 lo, hi;\n mov.b32 {lo, hi}, %2;\n cvt.rn.f16x2.e4m3x2 %0, lo;\n"
+      " cvt.rn.f16x2.e4m3x2 %1, hi;\n}"
+      : "=r"(d0), "=r"(d1)
+      : "r"(w));
+}
+__device__ __forceinline__ uint32_t hmul2_f16(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+// (lo, hi) floats -> packed fp16 pair, round to nearest even
+__device__ __forceinline__ uint32_t f16x2_pack(float lo, float hi) {
+  uint32_t d;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+  return d;
+}
+__device__ __forceinline__ uint32_t f16x2_splat(float x) { return f16x2_pack(x, x); }
+// packed bf16 pair -> packed fp16 pair
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
+  return f16x2_pack(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+// 1 when either half is an fp16 infinity or NaN
+__device__ __forceinline__ uint32_t f16x2_inf_bits(uint32_t d) {
+  return ((d & 0x7C00u) == 0x7C00u || (d & 0x7C000000u) == 0x7C000000u) ? 1u : 0u;
 }
 
 template <bool kFp8>
@@ -240,7 +261,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<kFp8>::kThreads,
 decode_pair_kernel(const __grid_constant__ CUtensorMap tm_cache,
                    const __grid_constant__ CUtensorMap tm_q, const PairArgs a) {
   constexpr int kStages = Cfg<kFp8>::kStages;
-  constexpr int kLand = Cfg<kFp8>::kLand > 0 ? Cfg<kFp8>::kLand : 1;  // the bf16 instance has none
   constexpr uint32_t kOffTmemPtr = Cfg<kFp8>::kOffTmemPtr;
   constexpr uint32_t kOffAbort = Cfg<kFp8>::kOffAbort;
   constexpr uint32_t kOffPM = Cfg<kFp8>::kOffPM;
@@ -269,16 +289,15 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_cache,
   if (threadIdx.x == 0) {
     *c.abort_flag = 0;
     for (int i = 0; i < kStages; ++i) {
-      // FP8: every converter warp of both CTAs arrives once per stage
-      mbar_init(c.bar(B_FULL0 + i), kFp8 ? 2 * kConvWarps : 1);
+      // FP8: the converter warp that owns the stage arrives, in both CTAs
+      mbar_init(c.bar(B_FULL0 + i), kFp8 ? 2 : 1);
       mbar_init(c.bar(B_EMPTY0 + i), 1);
     }
-    for (int i = 0; i < kLand; ++i) {
-      mbar_init(c.bar(B_LFULL0 + i), 1);
-      mbar_init(c.bar(B_LEMPTY0 + i), kConvWarps);
-    }
+    if (kFp8)
+      for (int i = 0; i < kStages; ++i) mbar_init(c.bar(B_LFULL0 + i), 1);
     mbar_init(c.bar(B_QFULL), 1);
     mbar_init(c.bar(B_QEMPTY), 1);
+    mbar_init(c.bar(B_QCONV), 2 * kConvWarps);
     mbar_init(c.bar(B_SFULL0), 1);
     mbar_init(c.bar(B_SFULL1), 1);
     mbar_init(c.bar(B_SFREE0), 16);
@@ -304,7 +323,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_cache,
   const int i0 = cta_begin[list], i1 = cta_begin[list + 1];
 
   const uint32_t q_s = base + kOffQ, p_s = base + kOffP, ring = base + kOffRing;
-  const uint32_t land_s = base + Cfg<kFp8>::kOffLand;
+  const uint32_t scale_s = base + Cfg<kFp8>::kOffScale;
   // barriers of the even CTA, as seen from this CTA
   const uint32_t lead_full0 = mapa_shared(c.bar(B_FULL0), 0);
   const uint32_t lead_qfull = mapa_shared(c.bar(B_QFULL), 0);
@@ -328,187 +347,267 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_cache,
   };
 
   if (kFp8 && warp == kProducerWarp) {
-    // ---------------------------------------- FP8 landing producer ---
+    // ------------------------------------------------ FP8 producer ---
+    // The same stage sequence as the bf16 producer, every load to this CTA's
+    // own barriers. Score chunks 2g and 2g+1 come as a pair of stages: the
+    // CTA's two pages' code columns [128 g, +128) (128-byte swizzle) land in
+    // the first stage, which the converters expand into both; the RoPE stage
+    // gets the pages' bf16 k^R as it is; an output stage gets one page's
+    // code columns in its upper half. Code stages also get the pages' token
+    // scales in the stage's scale slot. Every stage's landing barrier
+    // completes once per use (a pair's second stage by a plain arrive).
     if (lane == 0) {
       tma_prefetch_desc(&tm_cache);
       tma_prefetch_desc(&tm_q);
-      uint32_t lc = 0, ic = 0, q_armed = 0;
+      uint32_t sg = 0, ic = 0, q_armed = 0;
       bool ok = true;
-      // one landing slot: 64 rows x 128 bytes of the page at byte column x
-      // (+ the page's 64 scales)
-      auto land = [&](int x, int id, bool with_scales) -> bool {
-        const uint32_t l = lc % kLand;
-        if (lc >= kLand && !wait_fast(c, c.bar(B_LEMPTY0 + l), ((lc / kLand) - 1) & 1, false))
-          return false;
-        const uint32_t dst = land_s + l * kLandStride;
-        mbar_arrive_expect_tx(c.bar(B_LFULL0 + l), kBox + (with_scales ? 256u : 0u));
-        tma_load_2d(dst, &tm_cache, x, id * 64, c.bar(B_LFULL0 + l));
-        if (with_scales) bulk_load(dst + kBox, a.scales + (size_t)id * 64, 256, c.bar(B_LFULL0 + l));
-        ++lc;
-        return true;
+      auto acquire = [&](uint32_t seq, uint32_t &stg) -> bool {
+        stg = seq % kStages;
+        return seq < (uint32_t)kStages ||
+               wait_fast(c, c.bar(B_EMPTY0 + stg), ((seq / kStages) - 1) & 1, false);
       };
       for (int it = i0; it < i1 && ok; ++it, ++ic) {
         const WorkItem wi = items[it];
         const int T = tiles_of(wi.page_end - wi.page_begin);
         if (ic > 0 && !wait_bar(c, c.bar(B_QEMPTY), (ic - 1) & 1, false)) { ok = false; break; }
-        if (leader) {
-          mbar_arrive_expect_tx(c.bar(B_QFULL), 2 * kChunksQK * kBox);
-          ++q_armed;
-        }
+        // this CTA's 64 query rows, to its own barrier (the converters make
+        // the latent part fp16 before the MMA issuer sees it)
+        mbar_arrive_expect_tx(c.bar(B_QFULL), kChunksQK * kBox);
+        ++q_armed;
         const int tq = wi.b * a.q_len + wi.j;
         for (int ch = 0; ch < kChunksQK; ++ch)
-          tma_load_3d_pair(q_s + ch * kBox, &tm_q, 64 * ch, 64 * (int)rank, tq, lead_qfull);
+          tma_load_3d(q_s + ch * kBox, &tm_q, 64 * ch, 64 * (int)rank, tq, c.bar(B_QFULL));
         int ids_prev[kTilePages], ids_cur[kTilePages];
-        auto land_qk = [&](const int (&ids)[kTilePages]) -> bool {
-          for (int g = 0; g < 4; ++g)
-            for (int e = 0; e < 2; ++e)
-              if (ids[2 * rank + e] != -2 && !land(128 * g, ids[2 * rank + e], true)) return false;
-          for (int e = 0; e < 2; ++e)
-            if (ids[2 * rank + e] != -2 && !land(MLA_D_C, ids[2 * rank + e], false)) return false;
+        // this CTA's two pages of tile u (codes, k^R and scales) into L2
+        auto prefetch_tile = [&](int u) {
+          if (u >= T) return;
+          int ids[kTilePages];
+          tile_pages(wi, u, false, ids);
+          for (int e = 0; e < 2; ++e) {
+            const int id = ids[2 * rank + e];
+            if (id < 0) continue;
+            bulk_prefetch_l2(a.fp8_pool + (size_t)id * 64 * kFp8RowBytes, 64 * kFp8RowBytes);
+            bulk_prefetch_l2(a.scales + (size_t)id * 64, 256);
+          }
+        };
+        for (int u = 0; u < kFp8PrefetchTiles; ++u) prefetch_tile(u);
+        auto load_qk = [&](const int (&ids)[kTilePages]) -> bool {
+          const int id0 = ids[2 * rank], id1 = ids[2 * rank + 1];
+          const uint32_t npres = (id0 != -2 ? 1u : 0u) + (id1 != -2 ? 1u : 0u);
+          for (int g = 0; g < (kChunksQK - 1) / 2; ++g, sg += 2) {
+            uint32_t s0, s1;
+            if (!acquire(sg, s0) || !acquire(sg + 1, s1)) return false;
+            const uint32_t bar = c.bar(B_LFULL0 + s0);
+            mbar_arrive_expect_tx(bar, npres * (kBox + 256));
+            for (int e = 0; e < 2; ++e) {
+              const int id = e ? id1 : id0;
+              if (id == -2) continue;
+              tma_load_2d(ring + s0 * kStageBytes + e * kBox, &tm_cache, 128 * g, id * 64, bar);
+              bulk_load(scale_s + s0 * kScaleSlot + e * 256, a.scales + (size_t)id * 64, 256, bar);
+            }
+            mbar_arrive(c.bar(B_LFULL0 + s1));
+          }
+          uint32_t st;
+          if (!acquire(sg, st)) return false;
+          const uint32_t bar = c.bar(B_LFULL0 + st);
+          mbar_arrive_expect_tx(bar, npres * kBox);
+          for (int e = 0; e < 2; ++e) {
+            const int id = e ? id1 : id0;
+            if (id != -2) tma_load_2d(ring + st * kStageBytes + e * kBox, &tm_cache, MLA_D_C,
+                                      id * 64, bar);
+          }
+          ++sg;
           return true;
         };
-        auto land_pv = [&](const int (&ids)[kTilePages]) -> bool {
+        auto load_pv = [&](const int (&ids)[kTilePages]) -> bool {
           for (int j = 0; j < 2; ++j)
-            for (int p = 0; p < kTilePages; ++p)
-              if (ids[p] != -2 && !land(128 * (2 * j + (int)rank), ids[p], true)) return false;
+            for (int p = 0; p < kTilePages; ++p) {
+              if (ids[p] == -2) continue;
+              uint32_t stg;
+              if (!acquire(sg, stg)) return false;
+              const uint32_t st = ring + stg * kStageBytes, bar = c.bar(B_LFULL0 + stg);
+              mbar_arrive_expect_tx(bar, kHalfStage + 256);
+              tma_load_2d(st + kHalfStage, &tm_cache, 256 * j + 128 * (int)rank, ids[p] * 64, bar);
+              bulk_load(scale_s + stg * kScaleSlot, a.scales + (size_t)ids[p] * 64, 256, bar);
+              ++sg;
+            }
           return true;
         };
         for (int t = 0; t < T && ok; ++t) {
           tile_pages(wi, t, true, ids_cur);
-          if (!land_qk(ids_cur)) { ok = false; break; }
-          if (t >= 1 && !land_pv(ids_prev)) { ok = false; break; }
+          if (kFp8PrefetchTiles > 0) prefetch_tile(t + kFp8PrefetchTiles);
+          if (!load_qk(ids_cur)) { ok = false; break; }
+          if (t >= 1 && !load_pv(ids_prev)) { ok = false; break; }
 #pragma unroll
           for (int p = 0; p < kTilePages; ++p) ids_prev[p] = ids_cur[p];
         }
-        if (ok && !land_pv(ids_prev)) ok = false;
+        if (ok && !load_pv(ids_prev)) ok = false;
       }
-      // drain: every landing load completes on this CTA's own barriers
+      // drain: every load completes on this CTA's own barriers
       bool drained = true;
-      for (uint32_t k = lc > (uint32_t)kLand ? lc - kLand : 0; k < lc && drained; ++k)
-        drained = wait_drain(c, c.bar(B_LFULL0 + k % kLand), (k / kLand) & 1);
-      if (leader && q_armed && drained) wait_drain(c, c.bar(B_QFULL), (q_armed - 1) & 1);
+      for (uint32_t k = sg > (uint32_t)kStages ? sg - kStages : 0; k < sg && drained; ++k)
+        drained = wait_drain(c, c.bar(B_LFULL0 + k % kStages), (k / kStages) & 1);
+      if (q_armed && drained) wait_drain(c, c.bar(B_QFULL), (q_armed - 1) & 1);
     }
   } else if (kFp8 && warp >= kConvWarp0) {
     // ------------------------------------------------ FP8 converters ---
-    // Walk the same stage sequence as the MMA issuer and the same landing
-    // sequence as the producer; write bf16 operand stages (128-byte
-    // swizzle) from the E4M3 landing slots, times each token's scale.
-    const int ci = threadIdx.x - 32 * kConvWarp0;   // 0..kConvThreads-1
+    // Walk the MMA issuer's stage sequence in units: a score chunk pair, the
+    // RoPE stage, an output stage. Converter warp w owns the units whose
+    // number is w modulo kConvWarps and expands each alone: wait for its
+    // loads, then 16 rows at a time read the rows' codes into registers and
+    // write their fp16 values (times each token's scale; 128-byte swizzle),
+    // and hand the unit's stages to the MMA issuer. A row's fp16 values
+    // overwrite only that row's own codes, so a batch reads before it writes
+    // and no warp waits for another.
+    const int cw = warp - kConvWarp0;
     const uint32_t lead_full = leader ? c.bar(B_FULL0) : lead_full0;
-    uint32_t sg = 0, lc = 0;
-    bool ok = true;
-    auto take_stage = [&](uint32_t &stg) -> bool {
-      stg = sg % kStages;
-      return sg < (uint32_t)kStages ||
-             wait_warp(c, c.bar(B_EMPTY0 + stg), ((sg / kStages) - 1) & 1, false);
+    const uint32_t lead_qconv = mapa_shared(c.bar(B_QCONV), 0);
+    uint32_t sg = 0, ic = 0, un = 0;
+    bool ok = true, range_bad = false;
+    auto landed = [&](uint32_t seq, uint32_t &stg) -> bool {
+      stg = seq % kStages;
+      return wait_warp(c, c.bar(B_LFULL0 + stg), (seq / kStages) & 1, false);
     };
-    auto give_stage = [&](uint32_t stg) {
-      fence_proxy_async_smem();
-      __syncwarp();
+    auto arrive_full = [&](uint32_t seq) {
       if (lane == 0) {
         if (leader)
-          mbar_arrive(lead_full + 8 * stg);
+          mbar_arrive(lead_full + 8 * (seq % kStages));
         else
-          mbar_arrive_remote(lead_full + 8 * stg);
+          mbar_arrive_remote(lead_full + 8 * (seq % kStages));
       }
-      ++sg;
     };
-    auto wait_land = [&](uint32_t k) {
-      return wait_warp(c, c.bar(B_LFULL0 + k % kLand), (k / kLand) & 1, false);
+    auto mine = [&]() { return (int)(un++ % kConvWarps) == cw; };
+    // 16 codes of one token -> 16 fp16 values code * scale (exact for scales
+    // in [2^-15, 2^7]: the products are on the fp16 grid; larger scales can
+    // overflow and are reported)
+    // (Integer bit placement of the codes, code * 2^-8 then times scale *
+    // 2^8, measured slower than the conversion instruction, alone or for
+    // half the codes: 201 and 186 against 174 us on the 64 x 4096 workload.)
+    auto expand16 = [&](const uint4 &v, float sc, uint4 &o0, uint4 &o1) {
+      range_bad |= sc > 128.f;
+      const uint32_t s2 = f16x2_splat(sc);
+      uint32_t d[8];
+      e4m3x4_to_f16x2(v.x, d[0], d[1]);
+      e4m3x4_to_f16x2(v.y, d[2], d[3]);
+      e4m3x4_to_f16x2(v.z, d[4], d[5]);
+      e4m3x4_to_f16x2(v.w, d[6], d[7]);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) d[i] = hmul2_f16(d[i], s2);
+      o0 = make_uint4(d[0], d[1], d[2], d[3]);
+      o1 = make_uint4(d[4], d[5], d[6], d[7]);
     };
-    auto free_land = [&](uint32_t k) {
-      __syncwarp();
-      if (lane == 0) mbar_arrive(c.bar(B_LEMPTY0 + k % kLand));
+    // Rows [r_begin, r_end) of 128 codes (128-byte swizzle) at `src` + row *
+    // 128, scales at `sc_s` + row * 4: codes [0, 64) of a row go to `dst0`,
+    // [64, 128) to `dst1` (both 64 fp16 a row, 128-byte swizzle). When dst0
+    // or dst1 is src, each row overwrites only itself.
+    auto expand_rows = [&](uint32_t src, uint32_t sc_s, uint32_t dst0, uint32_t dst1,
+                           int r_begin, int r_end) {
+#pragma unroll 1
+      for (int r0 = r_begin; r0 < r_end; r0 += 16) {
+        uint4 v[4];
+        float sc[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int U = 32 * k + lane, t = r0 + (U >> 3), u = U & 7;
+          v[k] = lds128(src + t * 128 + ((u ^ (t & 7)) << 4));
+          sc[k] = lds_f32(sc_s + 4 * t);
+        }
+        __syncwarp();
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int U = 32 * k + lane, t = r0 + (U >> 3), u = U & 7, sw = t & 7;
+          uint4 o0, o1;
+          expand16(v[k], sc[k], o0, o1);
+          const uint32_t row = ((u >> 2) ? dst1 : dst0) + t * 128;
+          const int lu = 2 * (u & 3);
+          sts128(row + ((lu ^ sw) << 4), o0);
+          sts128(row + (((lu + 1) ^ sw) << 4), o1);
+        }
+        __syncwarp();
+      }
     };
-    auto slot = [&](uint32_t k) { return land_s + (k % kLand) * kLandStride; };
-    for (int it = i0; it < i1 && ok; ++it) {
+    auto conv_pv = [&](const int (&ids)[kTilePages]) -> bool {
+      for (int j = 0; j < 2; ++j)
+        for (int p = 0; p < kTilePages; ++p) {
+          if (ids[p] == -2) continue;
+          const uint32_t seq = sg++;
+          if (!mine()) continue;
+          uint32_t stg;
+          if (!landed(seq, stg)) return false;
+          // one page: the second 64-column box of row t is row t's codes
+          const uint32_t st = ring + stg * kStageBytes;
+          expand_rows(st + kHalfStage, scale_s + stg * kScaleSlot, st, st + kBox, 0, 64);
+          fence_proxy_async_smem();
+          __syncwarp();
+          arrive_full(seq);
+        }
+      return true;
+    };
+    for (int it = i0; it < i1 && ok; ++it, ++ic) {
       const WorkItem wi = items[it];
       const int T = tiles_of(wi.page_end - wi.page_begin);
-      int ids_prev[kTilePages], ids_cur[kTilePages];
-      auto conv_pv = [&](const int (&ids)[kTilePages]) -> bool {
-        for (int j = 0; j < 2; ++j)
-          for (int p = 0; p < kTilePages; ++p) {
-            if (ids[p] == -2) continue;
-            uint32_t stg;
-            if (!wait_land(lc) || !take_stage(stg)) return false;
-            const uint32_t src = slot(lc), dst = ring + stg * kStageBytes;
+      // the item's latent query columns (chunks 0-7) to fp16, a quarter per
+      // warp; the RoPE chunk stays bf16
+      {
+        if (!wait_warp(c, c.bar(B_QFULL), ic & 1, false)) { ok = false; break; }
+        constexpr int kQUnits = (kChunksQK - 1) * (int)kBox / 16 / kConvWarps;
+        uint32_t bad = 0;
+        const uint32_t q0 = q_s + 16 * kQUnits * cw;
 #pragma unroll 4
-            for (int k = 0; k < 512 / kConvThreads; ++k) {
-              const int U = ci + kConvThreads * k, t = U >> 3, u = U & 7, sw = t & 7;
-              const uint4 v = lds128(src + t * 128 + ((u ^ sw) << 4));
-              uint4 o0, o1;
-              fp8x16_to_bf16(v, lds_f32(src + kBox + 4 * t), o0, o1);
-              const uint32_t row = dst + (u >> 2) * kBox + t * 128;
-              const int lu = 2 * (u & 3);
-              sts128(row + ((lu ^ sw) << 4), o0);
-              sts128(row + (((lu + 1) ^ sw) << 4), o1);
-            }
-            give_stage(stg);
-            free_land(lc);
-            ++lc;
-          }
-        return true;
-      };
+        for (int k = lane; k < kQUnits; k += 32) {
+          const uint4 v = lds128(q0 + 16 * k);
+          const uint4 o = make_uint4(bf16x2_to_f16x2(v.x), bf16x2_to_f16x2(v.y),
+                                     bf16x2_to_f16x2(v.z), bf16x2_to_f16x2(v.w));
+          bad |= f16x2_inf_bits(o.x) | f16x2_inf_bits(o.y) | f16x2_inf_bits(o.z) |
+                 f16x2_inf_bits(o.w);
+          sts128(q0 + 16 * k, o);
+        }
+        range_bad |= bad != 0;
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          if (leader)
+            mbar_arrive(c.bar(B_QCONV));
+          else
+            mbar_arrive_remote(lead_qconv);
+        }
+      }
+      int ids_prev[kTilePages], ids_cur[kTilePages];
       for (int t = 0; t < T && ok; ++t) {
         tile_pages(wi, t, false, ids_cur);
         const bool pres[2] = {ids_cur[2 * rank] != -2, ids_cur[2 * rank + 1] != -2};
-        // score chunks 2g, 2g+1 from group g of the CTA's two pages
-        for (int g = 0; g < 4 && ok; ++g) {
-          const uint32_t k0 = lc, k1 = lc + (pres[0] ? 1 : 0);
-          lc += (pres[0] ? 1 : 0) + (pres[1] ? 1 : 0);
-          if ((pres[0] && !wait_land(k0)) || (pres[1] && !wait_land(k1))) { ok = false; break; }
-          for (int h = 0; h < 2; ++h) {
-            uint32_t stg;
-            if (!take_stage(stg)) { ok = false; break; }
-            const uint32_t dst = ring + stg * kStageBytes;
-#pragma unroll 4
-            for (int k = 0; k < 512 / kConvThreads; ++k) {
-              const int U = ci + kConvThreads * k, e = U >> 8, t = (U >> 2) & 63, uu = U & 3,
-                        sw = t & 7;
-              if (!pres[e]) continue;
-              const uint32_t src = slot(e ? k1 : k0);
-              const int u = 4 * h + uu;
-              const uint4 v = lds128(src + t * 128 + ((u ^ sw) << 4));
-              uint4 o0, o1;
-              fp8x16_to_bf16(v, lds_f32(src + kBox + 4 * t), o0, o1);
-              const uint32_t row = dst + e * kBox + t * 128;
-              sts128(row + (((2 * uu) ^ sw) << 4), o0);
-              sts128(row + (((2 * uu + 1) ^ sw) << 4), o1);
-            }
-            give_stage(stg);
+        // score chunk pairs: page e's codes at e * 8 KB of the first stage
+        for (int g = 0; g < (kChunksQK - 1) / 2; ++g, sg += 2) {
+          if (!mine()) continue;
+          uint32_t s0;
+          if (!landed(sg, s0)) { ok = false; break; }
+          const uint32_t s1 = (sg + 1) % kStages;
+          for (int e = 0; e < 2; ++e) {
+            if (!pres[e]) continue;
+            const uint32_t src = ring + s0 * kStageBytes + e * kBox;
+            expand_rows(src, scale_s + s0 * kScaleSlot + e * 256, src,
+                        ring + s1 * kStageBytes + e * kBox, 0, 64);
           }
-          if (!ok) break;
-          if (pres[0]) free_land(k0);
-          if (pres[1]) free_land(k1);
+          fence_proxy_async_smem();
+          __syncwarp();
+          arrive_full(sg);
+          arrive_full(sg + 1);
         }
         if (!ok) break;
-        // the RoPE chunk: bf16 rows copied unit by unit (same swizzle)
-        {
-          const uint32_t k0 = lc, k1 = lc + (pres[0] ? 1 : 0);
-          lc += (pres[0] ? 1 : 0) + (pres[1] ? 1 : 0);
-          uint32_t stg;
-          if ((pres[0] && !wait_land(k0)) || (pres[1] && !wait_land(k1)) || !take_stage(stg)) {
-            ok = false;
-            break;
-          }
-          const uint32_t dst = ring + stg * kStageBytes;
-#pragma unroll 4
-          for (int k = 0; k < 1024 / kConvThreads; ++k) {
-            const int U = ci + kConvThreads * k, e = U >> 9, t = (U >> 3) & 63, u = U & 7;
-            if (!pres[e]) continue;
-            const int off = t * 128 + ((u ^ (t & 7)) << 4);
-            sts128(dst + e * kBox + off, lds128(slot(e ? k1 : k0) + off));
-          }
-          give_stage(stg);
-          if (pres[0]) free_land(k0);
-          if (pres[1]) free_land(k1);
+        // the RoPE stage: the pages' bf16 k^R as landed
+        if (mine()) {
+          uint32_t st;
+          if (!landed(sg, st)) { ok = false; break; }
+          arrive_full(sg);
         }
+        ++sg;
         if (t >= 1 && !conv_pv(ids_prev)) { ok = false; break; }
 #pragma unroll
         for (int p = 0; p < kTilePages; ++p) ids_prev[p] = ids_cur[p];
       }
       if (ok && !conv_pv(ids_prev)) ok = false;
     }
+    if (__any_sync(0xffffffffu, range_bad) && lane == 0) report(a.status, MLA_DEV_RANGE);
   } else if (!kFp8 && warp == kProducerWarp) {
     if (lane == 0) {
       tma_prefetch_desc(&tm_cache);
@@ -602,8 +701,11 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_cache,
     }
   } else if (warp == kMmaWarp) {
     if (leader && lane == 0) {
-      constexpr uint32_t idesc_qk = idesc_bf16(128, 256, 0, 0);
-      constexpr uint32_t idesc_pv = idesc_bf16(128, 256, 0, 1);
+      // the FP8 instance's latent operands are fp16 (converted), its RoPE
+      // chunk and every operand of the bf16 instance bf16
+      constexpr uint32_t idesc_qk = idesc_f16kind(128, 256, 0, 0, !kFp8);
+      constexpr uint32_t idesc_qr = idesc_f16kind(128, 256, 0, 0, true);
+      constexpr uint32_t idesc_pv = idesc_f16kind(128, 256, 0, 1, !kFp8);
       uint32_t sg = 0, tg = 0, ic = 0, npv = 0;
       bool ok = true;
       auto take_stage = [&](uint32_t &stg) -> bool {
@@ -638,7 +740,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_cache,
         const WorkItem wi = items[it];
         const int np = wi.page_end - wi.page_begin;
         const int T = tiles_of(np);
-        if (!wait_bar(c, c.bar(B_QFULL), ic & 1, true)) { ok = false; break; }
+        if (!wait_bar(c, c.bar(kFp8 ? B_QCONV : B_QFULL), ic & 1, true)) { ok = false; break; }
         tc_fence_after();
         for (int t = 0; t < T; ++t, ++tg) {
           const int sb = tg & 1;
@@ -656,7 +758,8 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_cache,
             for (int kk = 0; kk < 4; ++kk) {
               const uint64_t ad = smem_desc(q_s + ch * kBox + kk * 32, 16, 1024, kSwizzle128B);
               const uint64_t bd = smem_desc(st + kk * 32, 16, 1024, kSwizzle128B);
-              mma_f16_ss_pair(d, ad, bd, idesc_qk, (ch | kk) ? 1u : 0u);
+              mma_f16_ss_pair(d, ad, bd, ch == kChunksQK - 1 ? idesc_qr : idesc_qk,
+                              (ch | kk) ? 1u : 0u);
             }
             mma_commit_pair(c.bar(B_EMPTY0 + stg));
           }
@@ -761,12 +864,24 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_cache,
 #pragma unroll
           for (int i = 0; i < 32; ++i) pk[i] = 0u;
         } else {
+          if constexpr (kFp8) {
+            // fp16 probabilities (p <= 2^8 under the lazy rescale); the sum
+            // takes the unrounded values
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const uint32_t p0 = rne_bf16_hi(ex2_approx(u2f(r[2 * i]) - m_ref));
-            const uint32_t p1 = rne_bf16_hi(ex2_approx(u2f(r[2 * i + 1]) - m_ref));
-            pk[i] = pack_hi_pair(p0, p1);
-            ls4[i & 3] += u2f(p0) + u2f(p1);  // the weights P*V uses
+            for (int i = 0; i < 32; ++i) {
+              const float p0 = ex2_approx(u2f(r[2 * i]) - m_ref);
+              const float p1 = ex2_approx(u2f(r[2 * i + 1]) - m_ref);
+              pk[i] = f16x2_pack(p0, p1);
+              ls4[i & 3] += p0 + p1;
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const uint32_t p0 = rne_bf16_hi(ex2_approx(u2f(r[2 * i]) - m_ref));
+              const uint32_t p1 = rne_bf16_hi(ex2_approx(u2f(r[2 * i + 1]) - m_ref));
+              pk[i] = pack_hi_pair(p0, p1);
+              ls4[i & 3] += u2f(p0) + u2f(p1);  // the weights P*V uses
+            }
           }
         }
         lsum = lsum * alpha + ((ls4[0] + ls4[1]) + (ls4[2] + ls4[3]));
@@ -947,8 +1062,9 @@ static mla_status_t launch_pair(const DecodeArgs &a, cudaStream_t stream) {
   const PlanHeader *ph = a.plan_host;
   if (ph->num_items == 0 || ph->num_ctas == 0) return MLA_OK;
   CUtensorMap tm_cache, tm_q;
-  mla_status_t st = kFp8 ? make_fp8_cache_map(&tm_cache, a.cache, (uint64_t)a.num_pages * MLA_PAGE)
-                         : make_cache_map(&tm_cache, a.cache, (uint64_t)a.num_pages * MLA_PAGE);
+  const uint64_t rows = (uint64_t)a.num_pages * MLA_PAGE;
+  mla_status_t st = kFp8 ? make_fp8_cache_map(&tm_cache, a.cache, rows)
+                         : make_cache_map(&tm_cache, a.cache, rows);
   if (st != MLA_OK) return st;
   st = make_query_map(&tm_q, a.q_full, a.batch * a.q_len, a.n_h);
   if (st != MLA_OK) return st;
@@ -968,6 +1084,7 @@ static mla_status_t launch_pair(const DecodeArgs &a, cudaStream_t stream) {
   t.wait_ns = g_wait_ns;
   t.suppress_arrive = g_suppress_arrive;
   t.scales = a.fp8_scales;
+  t.fp8_pool = kFp8 ? reinterpret_cast<const unsigned char *>(a.cache) : nullptr;
   // the shared-memory opt-in is a per-device attribute: set it once per device
   static std::mutex mu;
   static bool set[64] = {};

@@ -141,6 +141,11 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_
       : "memory");
 }
 
+// Bring [ptr, ptr + bytes) into L2 (16-byte aligned, bytes a multiple of 16).
+__device__ __forceinline__ void bulk_prefetch_l2(const void *ptr, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(ptr), "r"(bytes) : "memory");
+}
+
 __device__ __forceinline__ void tma_prefetch_desc(const void *tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
 }
@@ -324,6 +329,17 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_
          | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
          ((uint32_t)(N >> 3) << 17)      // N / 8
          | ((uint32_t)(M >> 4) << 24);   // M / 16
+}
+
+// The same for kind::f16 with fp16 (ab_bf16 = false) or bf16 A and B.
+__host__ __device__ constexpr uint32_t idesc_f16kind(int M, int N, int a_mn, int b_mn,
+                                                     bool ab_bf16) {
+  return (1u << 4)                                       // D format: f32
+         | ((ab_bf16 ? 1u : 0u) << 7)                    // A format: f16 / bf16
+         | ((ab_bf16 ? 1u : 0u) << 10)                   // B format: f16 / bf16
+         | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
+         ((uint32_t)(N >> 3) << 17)                      // N / 8
+         | ((uint32_t)(M >> 4) << 24);                   // M / 16
 }
 
 }  // namespace sm100

@@ -27,6 +27,7 @@ MLA_DEV_BAD_PAGE = 0x1
 MLA_DEV_BAD_POSITION = 0x2
 MLA_DEV_TIMEOUT = 0x4
 MLA_DEV_BAD_PLAN = 0x8
+MLA_DEV_RANGE = 0x10
 
 D_C, D_R, D_NOPE, D_V, ROW, PAGE = 512, 64, 128, 128, 576, 64
 MAX_Q_LEN = 1024

@@ -71,9 +71,14 @@ def test_decode_sources_hash_covers_the_decode_sources_only(tmp_path, monkeypatc
 
 def test_stored_traffic_figures_are_plausible():
     # every stored ncu traffic figure for v3 lies between the algorithmic
-    # bytes and 1.1x them (the decode reads each cache row once from HBM)
-    cache_bytes = 64 * 4096 * bench.ROW_BYTES
-    v3 = [t for (h, w), t in bench.TRAFFIC.items() if w == "v3"]
+    # bytes of its cache format and 1.1x them plus the outputs written (the
+    # decode reads each cache row once from HBM), and the current decode
+    # sources have a bf16 figure
+    row = {"bf16": bench.ROW_BYTES, "fp8": bench.FP8_TOKEN_BYTES}
+    out_bytes = 64 * 128 * (512 * 2 + 4)
+    v3 = [(cache, t) for (h, w, cache), t in bench.TRAFFIC.items() if w == "v3"]
     assert v3
-    for t in v3:
-        assert cache_bytes <= t <= math.ceil(1.1 * cache_bytes)
+    for cache, t in v3:
+        cache_bytes = 64 * 4096 * row[cache]
+        assert cache_bytes <= t <= math.ceil(1.1 * cache_bytes) + out_bytes
+    assert (bench.decode_sources_hash(), "v3", "bf16") in bench.TRAFFIC

@@ -130,3 +130,23 @@ def test_fp8_workload_full_size(dev, name):
     torch.cuda.synchronize()
     assert sess.read_status() == 0
     check_fp8(sess, inp, synth.sample_sequences(w, inp.lens, 6), table, whole_pool=False)
+
+
+@pytest.mark.parametrize("where", ["query", "latent"])
+def test_fp8_range_reported(dev, where):
+    # The FP8 decode computes in fp16: a query value beyond its range, or a
+    # token whose scale exceeds 2^7 (a latent value beyond 448 * 2^7), sets
+    # MLA_DEV_RANGE; in-range inputs leave the status clear (every other test)
+    lens = [300, 129]
+    w = synth.Workload("fp8range", B=len(lens), q_len=1, L=300, n_h=128, seed=31)
+    inp = synth.make_decode_inputs(w, lens=lens)
+    sess = DecodeSession(inp, dev, fp8=True)
+    if where == "latent":
+        sess.c_new[1, 7] = 1.0e5
+    sess.append()
+    sess.absorb()
+    if where == "query":
+        sess.q_full[0, 5, 11] = 1.0e5
+    sess.attend()
+    torch.cuda.synchronize()
+    assert sess.read_status() & mla.MLA_DEV_RANGE
