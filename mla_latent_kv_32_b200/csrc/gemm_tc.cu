@@ -63,7 +63,6 @@ struct GemmTcArgs {
   uint32_t *status;
   int tile_z;           // z extent of the GEMM tiles; CTAs beyond it run the side job
   int b_shared;         // every batch z reads the same B (its tensor map has one z slice)
-  int two_m;            // a CTA covers 256 rows of A: two 128-row accumulators
   float *part;          // fp32 output split over K: split s writes its partial tile at
                         // ((s * batch + z) * N + n) * M + m; a second kernel sums them
   // side job (rope_q_pe == nullptr: none)
@@ -155,6 +154,9 @@ __device__ __noinline__ bool wait_bar_g(uint32_t bar, uint32_t parity, uint32_t 
   }
 }
 
+// kTwoM: a CTA covers 256 rows of A with two 128-row accumulators (the
+// instances keep the one-accumulator loops free of the second's branches).
+template <bool kTwoM>
 __global__ void __launch_bounds__(128, 4)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                const GemmTcArgs g) {
@@ -179,8 +181,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__
   unsigned char *smem = smem_raw + (base - raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n0 = blockIdx.x * g.BN;
-  const int m0 = blockIdx.y * (g.two_m ? 256 : 128);
-  const uint32_t a_bytes = g.two_m ? 2 * kAStage : kAStage;
+  const int m0 = blockIdx.y * (kTwoM ? 256 : 128);
+  constexpr uint32_t a_bytes = kTwoM ? 2 * kAStage : kAStage;
   const int z = blockIdx.z / g.splits;
   const int split = blockIdx.z % g.splits;
   const int kc0 = split * g.k_chunks;
@@ -221,7 +223,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__
         tma_load_3d(a_s + 8192, &tm_a, m0 + 64, kc * 64, z, bar_full + 8 * s);
       } else {
         tma_load_3d(a_s, &tm_a, kc * 64, m0, z, bar_full + 8 * s);
-        if (g.two_m) tma_load_3d(a_s + kAStage, &tm_a, kc * 64, m0 + 128, z, bar_full + 8 * s);
+        if (kTwoM) tma_load_3d(a_s + kAStage, &tm_a, kc * 64, m0 + 128, z, bar_full + 8 * s);
       }
       tma_load_3d(b_s, &tm_b, kc * 64, n0, g.b_shared ? 0 : z, bar_full + 8 * s);
     }
@@ -240,7 +242,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__
                                    : smem_desc(a_s + kk * 32, 16, 1024, kSwizzle128B);
         const uint64_t bd = smem_desc(b_s + kk * 32, 16, 1024, kSwizzle128B);
         mma_f16_ss(tmem, ad, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
-        if (g.two_m)
+        if (kTwoM)
           mma_f16_ss(tmem + g.BN, smem_desc(a_s + kAStage + kk * 32, 16, 1024, kSwizzle128B), bd,
                      idesc, (i > 0 || kk > 0) ? 1u : 0u);
       }
@@ -253,22 +255,30 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__
   const bool done = wait_bar_g(bar_done, 0, g.status);
   tc_fence_after();
   const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-  for (int pass = 0; pass <= g.two_m; ++pass)
+#pragma unroll
+  for (int pass = 0; pass < (kTwoM ? 2 : 1); ++pass)
   for (int ch = 0; ch * 32 < g.BN; ++ch) {
     const int m = m0 + 128 * pass + threadIdx.x;
     uint32_t r[32];
     tmem_ld32(tmem + lane_off + pass * g.BN + 32 * ch, r);
     tmem_wait_ld();
     if (!done || kc1 <= kc0 || m >= g.M) continue;
+    if (g.part != nullptr) {
+      // this split's partial tile
+      float *dst = g.part + ((long long)split * g.batch + z) * g.N * g.M + m;
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const int n = n0 + 32 * ch + e;
+        if (n >= g.N) break;
+        dst[(long long)n * g.M] = __uint_as_float(r[e]);
+      }
+      continue;
+    }
 #pragma unroll
     for (int e = 0; e < 32; ++e) {
       const int n = n0 + 32 * ch + e;
       if (n >= g.N) break;
       const float v = __uint_as_float(r[e]);
-      if (g.part != nullptr) {
-        g.part[(((long long)split * g.batch + z) * g.N + n) * g.M + m] = v;
-        continue;
-      }
       if (g.ws != nullptr) {
         atomicAdd(g.ws + ((long long)z * g.N + n) * g.M + m, v);
         continue;
@@ -440,7 +450,6 @@ mla_status_t launch_gemm_tc(const GemmTcDesc &d, cudaStream_t stream) {
   g.splits = splits;
   g.k_chunks = (kchunks + splits - 1) / splits;
   g.stage_bytes = (two_m ? 2 : 1) * kAStage + (((uint32_t)BN * 128 + 1023u) & ~1023u);
-  g.two_m = two_m ? 1 : 0;
   // A grid that fits one CTA per SM keeps every k-chunk of a tile in flight
   // (up to kMaxStages, within the shared memory), so a tile waits one load
   // round trip rather than one per ring cycle; denser grids keep a shallower
@@ -488,10 +497,11 @@ mla_status_t launch_gemm_tc(const GemmTcDesc &d, cudaStream_t stream) {
       return fail(MLA_ERR_UNSUPPORTED, "split-K needs a contiguous fp32 output");
     MLA_CUDA_TRY(cudaMemsetAsync(d.C, 0, d.c_bytes, stream));
   }
-  MLA_CUDA_TRY(cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  auto kernel = two_m ? gemm_tc_kernel<true> : gemm_tc_kernel<false>;
+  MLA_CUDA_TRY(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     (int)smem_bytes));
   dim3 grid(ntile, mtile, d.batch * splits + side_z);
-  gemm_tc_kernel<<<grid, 128, smem_bytes, stream>>>(tm_a, tm_b, g);
+  kernel<<<grid, 128, smem_bytes, stream>>>(tm_a, tm_b, g);
   MLA_LAUNCH_CHECK("gemm_tc_kernel");
   if (pl.part) {
     const long long total = (long long)d.M * d.N * d.batch;
