@@ -357,7 +357,10 @@ def run_rows(args):
     """Each call of the path alone, L2 flushed before every call: time, its
     algorithmic bytes (weights and activations read once, outputs written
     once) and FLOPs, and the fraction of the roofline (the slower of bytes ÷
-    measured HBM bandwidth and FLOPs ÷ measured bf16 peak)."""
+    measured HBM bandwidth and FLOPs ÷ measured bf16 peak). Each call is
+    captured in a CUDA graph and timed as one replay: a call's host-side
+    argument checks and tensor-map encoding are not in the time, the replay's
+    own launch latency is."""
     import torch
     import synth
     from mla_latent_kv_32_b200 import build as build_mod
@@ -375,14 +378,20 @@ def run_rows(args):
     def timed(fn, K):
         for _ in range(3):
             fn()
+        side = torch.cuda.Stream()
+        side.wait_stream(stream)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=side):
+            fn(side)
+        stream.wait_stream(side)
         if args.ramp_seconds > 0:
-            ramp_clocks(lambda: (flush(), fn()), seconds=min(0.2, args.ramp_seconds))
+            ramp_clocks(lambda: (flush(), graph.replay()), seconds=min(0.2, args.ramp_seconds))
         ts = []
         for _ in range(K):
             flush()
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(stream)
-            fn()
+            graph.replay()
             b.record(stream)
             torch.cuda.synchronize()
             ts.append(a.elapsed_time(b) * 1e3)
