@@ -76,6 +76,33 @@ def test_empty_inputs_are_noops_without_a_device(lib):
     mla.mla_gemm_bf16(None, 64, None, 64, None, 64, 1, 64, 0, 64, stream=0)      # N = 0
     mla.mla_gemm_bf16_ws(None, 64, None, 64, None, 64, 0, 0, 64, 64, None, 0, stream=0)
     assert mla.mla_gemm_bf16_workspace_bytes(0, 64, 64) == 0
+    # the fused append + absorption with neither tokens to append nor queries
+    mla.mla_append_absorb_q(None, 1, None, 1, 1, None, None, None, 576, None, 576, 0, None, 24576,
+                            None, 24576, None, None, None, 1, 0, 128, None, stream=0)
+    # the FP8 cache's entry points, the folds and the folded absorption
+    mla.mla_cache_append_fp8(None, None, 1, None, 1, 1, None, None, None, 512, None, 64, None, 1,
+                             0, stream=0)
+    plan, _ = mla.mla_decode_plan(np.zeros(0, np.int32), 0, 1, 128, num_ctas=8)
+    mla.mla_decode_attention_fp8(None, None, None, 1, None, 1, 0, 1, 128, 0.07, plan, plan, None,
+                                 0, None, stream=0)
+    mla.mla_fold_qk(None, 1536, 1536, None, 0, None, None, 0, stream=0)
+    mla.mla_fold_o(None, 16384, 7168, None, 0, None, stream=0)
+    mla.mla_absorb_q_folded(None, 1536, 1536, None, 8192, None, None, None, 1, 0, 128, None,
+                            stream=0)
+
+
+def test_fused_append_absorb_checks_both_halves(lib):
+    """mla_append_absorb_q validates the append's and the absorption's
+    arguments before launching anything: a NULL cache with tokens to append,
+    or an unsupported head count with queries, fails on the host."""
+    with pytest.raises(mla.MlaError) as e:
+        mla.mla_append_absorb_q(None, 1, None, 1, 1, None, None, None, 576, None, 576, 4, None,
+                                24576, None, 24576, None, None, None, 1, 0, 128, None, stream=0)
+    assert e.value.status == mla.MLA_ERR_INVALID_ARGUMENT
+    with pytest.raises(mla.MlaError) as e:
+        mla.mla_append_absorb_q(None, 1, None, 1, 1, None, None, None, 576, None, 576, 0, 16,
+                                2048, 16, 1024, 16, None, None, 0, 1, 24, 16, stream=0)
+    assert e.value.status == mla.MLA_ERR_UNSUPPORTED
 
 
 def test_rope_table_matches_oracle(lib):
