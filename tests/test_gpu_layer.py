@@ -65,12 +65,14 @@ def test_layer(dev, name):
 
 @pytest.mark.parametrize("M,N,K,fp32", [
     (256, 576, 7168, 0), (256, 1536, 7168, 0), (7, 64, 512, 0), (256, 24576, 1536, 0),
-    (256, 7168, 16384, 1), (100, 1100, 640, 1), (3, 2048, 1024, 0)])
+    (256, 7168, 16384, 1), (100, 1100, 640, 1), (3, 2048, 1024, 0), (64, 24576, 512, 0),
+    (48, 20000, 512, 0)])
 def test_split_k_gemm_matches_fp32(dev, M, N, K, fp32):
     # C = X W^T with a workspace (split over K into partial sums when the tile
-    # grid is below one wave; 256-row weight tiles from 1024 rows up) and
-    # without one (fp32 outputs may split with atomic adds), against a float64
-    # product of the same bf16 inputs
+    # grid is below one wave; 256-row weight tiles from 1024 rows up, also
+    # with narrow token tiles, 64 x 24576 and 48 x 20000 here, the latter
+    # with a ragged last tile) and without one (fp32 outputs may split with
+    # atomic adds), against a float64 product of the same bf16 inputs
     g = torch.Generator().manual_seed(M * 7 + N)
     X = (torch.randn(M, K, generator=g) / math.sqrt(K)).to(torch.bfloat16)
     W = torch.randn(N, K, generator=g).to(torch.bfloat16)
