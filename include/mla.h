@@ -67,7 +67,7 @@ typedef enum mla_status {
 #define MLA_DEV_BAD_POSITION 0x2u /* position outside the RoPE table or the page table */
 #define MLA_DEV_TIMEOUT 0x4u      /* a bounded wait expired: the kernel abandoned its work */
 #define MLA_DEV_BAD_PLAN 0x8u     /* a work item disagrees with the sequence lengths */
-#define MLA_DEV_RANGE 0x10u       /* FP8 decode: a query or k^R value that is not finite in
+#define MLA_DEV_RANGE 0x10u       /* FP8 decode: a latent query value that is not finite in
                                      fp16 (|x| >= 65520, inf, NaN), or a token scale above 2^7 */
 
 /* Message of the last failed call on this thread ("" if none). */
@@ -312,7 +312,7 @@ mla_status_t mla_decode_attention_noalloc(const mla_bf16_t *q_full, const mla_bf
  * [2^-15, 2^7]; below 2^-15 the smallest codes round on the fp16 grid), the
  * query's latent columns as fp16 (exact for bf16 values in the fp16 normal
  * range), the probabilities rounded to fp16. The RoPE products stay bf16.
- * A query or k^R value that is not finite in fp16, or a scale above 2^7,
+ * A latent query value that is not finite in fp16, or a scale above 2^7,
  * sets MLA_DEV_RANGE in *status (the outputs are then not meaningful).
  */
 mla_status_t mla_cache_append_fp8(uint8_t *cache, float *scales, int num_pages,
