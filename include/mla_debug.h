@@ -45,6 +45,24 @@ mla_status_t mla_decode_attention_cudacore(const mla_bf16_t *q_full, const mla_b
  */
 mla_status_t mla_debug_decode_wait(double wait_cap_seconds, int suppress_arrive);
 
+/*
+ * mla_debug_gemm_plan -- host, no device needed. The tile plan the
+ * tensor-core GEMM takes for a problem, so that tests can check the planner
+ * on the CPU. C[z][m][n] = sum_k A[z][m][k] B[z][n][k] with M weight rows, N
+ * tokens, K the reduction, `batch` problems; a_mn: A is MN-major; c_fp32: the
+ * output is float32; fp32_part: an fp32 output with a partial-sum workspace
+ * (mla_gemm_bf16_ws); atomic_split: a split over K may accumulate with atomic
+ * adds; sms: the SM count to plan for.
+ *   out[0] N tile (BN), out[1] 128-row accumulators per CTA (1 or 2),
+ *   out[2] N tiles, out[3] M tiles, out[4] splits over K, out[5] 64-wide
+ *   k-chunks per split, out[6] 1 when the splits write partial tiles,
+ *   out[7] the partial-tile workspace bytes (low 31 bits are enough for the
+ *   checked shapes; larger values saturate at 2^31 - 1).
+ * Returns INVALID_ARGUMENT for non-positive sizes or a NULL `out`.
+ */
+mla_status_t mla_debug_gemm_plan(int M, int N, int K, int batch, int a_mn, int c_fp32,
+                                 int fp32_part, int atomic_split, int sms, int32_t *out);
+
 #ifdef __cplusplus
 }
 #endif

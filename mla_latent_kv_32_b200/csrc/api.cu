@@ -518,6 +518,24 @@ mla_status_t mla_cache_append_fp8(uint8_t *cache, float *scales, int num_pages,
                                  status, (cudaStream_t)stream);
 }
 
+mla_status_t mla_debug_gemm_plan(int M, int N, int K, int batch, int a_mn, int c_fp32,
+                                 int fp32_part, int atomic_split, int sms, int32_t *out) {
+  clear_error();
+  MLA_CHECK_ARG(out != nullptr, "NULL out");
+  MLA_CHECK_ARG(M > 0 && N > 0 && K > 0 && batch > 0 && sms > 0, "non-positive size");
+  const GemmPlan pl = plan_gemm(M, N, K, batch, a_mn != 0, c_fp32 != 0, fp32_part != 0,
+                                atomic_split != 0, sms);
+  out[0] = pl.BN;
+  out[1] = pl.two_m ? 2 : 1;
+  out[2] = pl.ntile;
+  out[3] = pl.mtile;
+  out[4] = pl.splits;
+  out[5] = pl.k_chunks;
+  out[6] = pl.part ? 1 : 0;
+  out[7] = (int32_t)std::min<size_t>(pl.part_bytes, 0x7FFFFFFF);
+  return MLA_OK;
+}
+
 mla_status_t mla_debug_decode_wait(double wait_cap_seconds, int suppress_arrive) {
   clear_error();
   return set_decode_wait(wait_cap_seconds, suppress_arrive);

@@ -65,6 +65,7 @@ SIGNATURES = {
     "mla_decode_attention": (_I, [_P, _P, _I, _P, _I, _I, _I, _I, _F, _P, _P, _P, _SZ, _P, _P,
                                   _P, _P]),
     "mla_debug_decode_wait": (_I, [ctypes.c_double, _I]),
+    "mla_debug_gemm_plan": (_I, [_I, _I, _I, _I, _I, _I, _I, _I, _I, _P]),
     "mla_decode_attention_cudacore": (_I, [_P, _P, _I, _P, _I, _I, _I, _I, _F, _P, _P, _P, _SZ,
                                            _P, _P, _P, _P]),
     "mla_decode_attention_noalloc": (_I, [_P, _P, _I, _P, _I, _I, _I, _I, _F, _P, _P, _P, _P,
@@ -190,6 +191,16 @@ def mla_debug_decode_wait(wait_cap_seconds: float = 1.0, suppress_arrive: int = 
     """Failure-detection switch of the tensor-core decode kernel (include/mla_debug.h)."""
     _check(load().mla_debug_decode_wait(float(wait_cap_seconds), int(suppress_arrive)),
            "mla_debug_decode_wait")
+
+
+def mla_debug_gemm_plan(M, N, K, batch=1, a_mn=0, c_fp32=0, fp32_part=0, atomic_split=0,
+                        sms=148) -> dict:
+    """The tensor-core GEMM's tile plan for a problem (include/mla_debug.h)."""
+    out = (ctypes.c_int32 * 8)()
+    _check(load().mla_debug_gemm_plan(M, N, K, batch, int(a_mn), int(c_fp32), int(fp32_part),
+                                      int(atomic_split), sms, out), "mla_debug_gemm_plan")
+    keys = ("BN", "accumulators", "ntile", "mtile", "splits", "k_chunks", "part", "part_bytes")
+    return dict(zip(keys, list(out)))
 
 
 def mla_decode_attention_cudacore(q_full, cache, num_pages, block_table, max_pages, batch, q_len,
