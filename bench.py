@@ -533,7 +533,7 @@ def measure_decode_config(name, dev, flush, stream, K, peaks, args, fp8=False):
            "plan": {"work_lists": int(sess.info.num_ctas), "items": int(sess.info.num_items),
                     "partials": int(sess.info.num_partials),
                     "combine": int(sess.info.num_combine)},
-           "launches_per_step": (4 if fp8 else 3) + (1 if sess.info.num_combine else 0)}
+           "launches_per_step": 3 + (1 if sess.info.num_combine else 0)}
     if w.q_len > 16:
         # the same attention in the expanded (non-absorbed) form: 2*(128+64)
         # + 2*128 FLOP per (visible token, head, query) plus expanding K^C and
@@ -810,11 +810,11 @@ def main():
         "peak_source": f"{peak_src} (MEASURED_PEAKS.json burst figures)"
         if peak_src == "measured" else "fallback", "sources": src_hash,
     }
-    # the absorb GEMM (with the q RoPE pack and the cache append in the same
-    # launch; the FP8 cache appends in its own launch), decode, [combine],
-    # out_absorb per timed step, plus decode [+ combine] per timed attention call
+    # the absorb GEMM (with the q RoPE pack and the cache append, bf16 or FP8,
+    # in the same launch), decode, [combine], out_absorb per timed step, plus
+    # decode [+ combine] per timed attention call
     combine = 1 if sess.info.num_combine > 0 else 0
-    per_step = (4 if fp8 else 3) + combine
+    per_step = 3 + combine
     launches_timed = K * per_step + K * (1 + combine)
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,

@@ -321,6 +321,22 @@ mla_status_t mla_cache_append_fp8(uint8_t *cache, float *scales, int num_pages,
                                   const mla_bf16_t *c_kv, int ld_c, const mla_bf16_t *k_pe,
                                   int ld_k, const float *rope_table, int max_pos, int n_tokens,
                                   uint32_t *status, mla_stream_t stream);
+/*
+ * mla_append_fp8_absorb_q -- device. mla_cache_append_fp8 and mla_absorb_q of
+ * one decode step in one launch, as mla_append_absorb_q is for the bf16
+ * cache: the same results as the two calls in that order; the cache arguments
+ * are those of mla_cache_append_fp8, the query arguments those of
+ * mla_absorb_q. Errors: as the two calls.
+ */
+mla_status_t mla_append_fp8_absorb_q(uint8_t *cache, float *scales, int num_pages,
+                                     const int32_t *block_table, int batch, int max_pages,
+                                     const int32_t *seq_idx, const int32_t *tok_pos,
+                                     const mla_bf16_t *c_kv, int ld_c, const mla_bf16_t *k_pe,
+                                     int ld_k, int n_tokens, const mla_bf16_t *q_nope, int ld_qn,
+                                     const mla_bf16_t *q_pe, int ld_qp, const mla_bf16_t *w_uk,
+                                     const int32_t *q_pos, const float *rope_table, int max_pos,
+                                     int T, int n_h, mla_bf16_t *q_full, uint32_t *status,
+                                     mla_stream_t stream);
 mla_status_t mla_decode_attention_fp8(const mla_bf16_t *q_full, const uint8_t *cache,
                                       const float *scales, int num_pages,
                                       const int32_t *block_table, int max_pages, int batch,

@@ -190,6 +190,66 @@ mla_status_t mla_append_absorb_q(mla_bf16_t *cache, int num_pages, const int32_t
   if (st != MLA_OK) return st;
   AppendJob app;
   app.cache = cache;
+  app.cache8 = nullptr;
+  app.scales8 = nullptr;
+  app.num_pages = num_pages;
+  app.block_table = block_table;
+  app.batch = batch;
+  app.max_pages = max_pages;
+  app.seq_idx = seq_idx;
+  app.pos = tok_pos;
+  app.c_kv = c_kv;
+  app.ld_c = ld_c;
+  app.k_pe = k_pe;
+  app.ld_k = ld_k;
+  app.n_tokens = n_tokens;
+  return launch_absorb_q(q_nope, ld_qn, q_pe, ld_qp, q_pos, rope_table, max_pos, w_uk, T, n_h,
+                         q_full, status, (cudaStream_t)stream, &app);
+}
+
+mla_status_t mla_append_fp8_absorb_q(uint8_t *cache, float *scales, int num_pages,
+                                     const int32_t *block_table, int batch, int max_pages,
+                                     const int32_t *seq_idx, const int32_t *tok_pos,
+                                     const mla_bf16_t *c_kv, int ld_c, const mla_bf16_t *k_pe,
+                                     int ld_k, int n_tokens, const mla_bf16_t *q_nope, int ld_qn,
+                                     const mla_bf16_t *q_pe, int ld_qp, const mla_bf16_t *w_uk,
+                                     const int32_t *q_pos, const float *rope_table, int max_pos,
+                                     int T, int n_h, mla_bf16_t *q_full, uint32_t *status,
+                                     mla_stream_t stream) {
+  clear_error();
+  MLA_CHECK_ARG(n_tokens >= 0 && T >= 0, "negative size");
+  if (T == 0)
+    return mla_cache_append_fp8(cache, scales, num_pages, block_table, batch, max_pages, seq_idx,
+                                tok_pos, c_kv, ld_c, k_pe, ld_k, rope_table, max_pos, n_tokens,
+                                status, stream);
+  if (n_tokens == 0)
+    return mla_absorb_q(q_nope, ld_qn, q_pe, ld_qp, w_uk, q_pos, rope_table, max_pos, T, n_h,
+                        q_full, status, stream);
+  // the append's arguments, as mla_cache_append_fp8 checks them
+  MLA_CHECK_ARG(cache && scales && block_table && seq_idx && tok_pos && c_kv && k_pe &&
+                    rope_table,
+                "NULL device pointer");
+  MLA_CHECK_ARG(num_pages > 0 && batch > 0 && max_pages > 0 && max_pos > 0,
+                "sizes must be positive");
+  MLA_CHECK_ARG(aligned16(cache) && aligned16(scales) && aligned16(c_kv) && aligned16(k_pe) &&
+                    aligned16(rope_table),
+                "cache, scales, c_kv, k_pe and rope_table must be 16-byte aligned");
+  MLA_CHECK_ARG(ld_c >= MLA_D_C && ld_c % 8 == 0, "ld_c must be >= 512 and a multiple of 8");
+  MLA_CHECK_ARG(ld_k >= MLA_D_R && ld_k % 8 == 0, "ld_k must be >= 64 and a multiple of 8");
+  // the absorption's, as mla_absorb_q checks them
+  if (!heads_supported(n_h))
+    return fail(MLA_ERR_UNSUPPORTED, "n_h = %d (supported: 16..128, multiple of 16)", n_h);
+  MLA_CHECK_ARG(q_nope && q_pe && w_uk && q_full, "NULL device pointer");
+  MLA_CHECK_ARG(aligned16(q_nope) && aligned16(q_pe) && aligned16(w_uk) && aligned16(q_full),
+                "pointers must be 16-byte aligned");
+  MLA_CHECK_ARG(ld_qn >= n_h * MLA_D_NOPE && ld_qn % 8 == 0, "ld_qn too small or unaligned");
+  MLA_CHECK_ARG(ld_qp >= n_h * MLA_D_R && ld_qp % 8 == 0, "ld_qp too small or unaligned");
+  mla_status_t st = require_sm100();
+  if (st != MLA_OK) return st;
+  AppendJob app;
+  app.cache = nullptr;
+  app.cache8 = cache;
+  app.scales8 = scales;
   app.num_pages = num_pages;
   app.block_table = block_table;
   app.batch = batch;

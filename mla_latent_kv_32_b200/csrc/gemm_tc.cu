@@ -168,11 +168,18 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__
     if (g.rope_q_pe != nullptr) rope_side_job(g, cta, ctas);
     // the step's cache append: one warp per token
     const int warps = ctas * (blockDim.x >> 5);
-    for (int t = cta * (blockDim.x >> 5) + (threadIdx.x >> 5); t < g.app.n_tokens; t += warps)
-      append_token_warp(g.app.cache, g.app.num_pages, g.app.block_table, g.app.batch,
-                        g.app.max_pages, g.app.seq_idx, g.app.pos, g.app.c_kv, g.app.ld_c,
-                        g.app.k_pe, g.app.ld_k, g.rope_table, g.rope_max_pos, t, threadIdx.x & 31,
-                        g.status);
+    for (int t = cta * (blockDim.x >> 5) + (threadIdx.x >> 5); t < g.app.n_tokens; t += warps) {
+      if (g.app.cache8 != nullptr)
+        append_token_fp8_warp(g.app.cache8, g.app.scales8, g.app.num_pages, g.app.block_table,
+                              g.app.batch, g.app.max_pages, g.app.seq_idx, g.app.pos, g.app.c_kv,
+                              g.app.ld_c, g.app.k_pe, g.app.ld_k, g.rope_table, g.rope_max_pos, t,
+                              threadIdx.x & 31, g.status);
+      else
+        append_token_warp(g.app.cache, g.app.num_pages, g.app.block_table, g.app.batch,
+                          g.app.max_pages, g.app.seq_idx, g.app.pos, g.app.c_kv, g.app.ld_c,
+                          g.app.k_pe, g.app.ld_k, g.rope_table, g.rope_max_pos, t,
+                          threadIdx.x & 31, g.status);
+    }
     return;
   }
   extern __shared__ __align__(1024) unsigned char smem_raw[];

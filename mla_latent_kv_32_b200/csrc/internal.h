@@ -10,7 +10,9 @@ namespace mla {
 // (the absorption GEMM): n_tokens == 0 means none. Same arguments as
 // mla_cache_append.
 struct AppendJob {
-  uint16_t *cache;
+  uint16_t *cache;      // bf16 cache, or NULL with the FP8 cache below
+  uint8_t *cache8;      // FP8 cache rows (640 bytes) and their scales, or NULL
+  float *scales8;
   int num_pages;
   const int32_t *block_table;
   int batch, max_pages;

@@ -85,6 +85,8 @@ SIGNATURES = {
                                       _P, _P, _P, _P]),
     "mla_append_absorb_q": (_I, [_P, _I, _P, _I, _I, _P, _P, _P, _I, _P, _I, _I, _P, _I, _P, _I,
                                  _P, _P, _P, _I, _I, _I, _P, _P, _P]),
+    "mla_append_fp8_absorb_q": (_I, [_P, _P, _I, _P, _I, _I, _P, _P, _P, _I, _P, _I, _I, _P,
+                                     _I, _P, _I, _P, _P, _P, _I, _I, _I, _P, _P, _P]),
     "mla_fold_qk_workspace_bytes": (_SZ, [_I]),
     "mla_fold_qk": (_I, [_P, _I, _I, _P, _I, _P, _P, _SZ, _P]),
     "mla_fold_o": (_I, [_P, _I, _I, _P, _I, _P, _P]),
@@ -318,6 +320,19 @@ def mla_decode_attention_fp8(q_full, cache, scales, num_pages, block_table, max_
                                            _ptr(workspace), workspace_bytes, _ptr(o_latent),
                                            _ptr(lse), _ptr(status), _stream(stream)),
            "mla_decode_attention_fp8")
+
+
+def mla_append_fp8_absorb_q(cache, scales, num_pages, block_table, batch, max_pages, seq_idx,
+                            tok_pos, c_kv, ld_c, k_pe, ld_k, n_tokens, q_nope, ld_qn, q_pe, ld_qp,
+                            w_uk, q_pos, rope_table, max_pos, T, n_h, q_full, status=None,
+                            stream=None):
+    _check(load().mla_append_fp8_absorb_q(_ptr(cache), _ptr(scales), num_pages,
+                                          _ptr(block_table), batch, max_pages, _ptr(seq_idx),
+                                          _ptr(tok_pos), _ptr(c_kv), ld_c, _ptr(k_pe), ld_k,
+                                          n_tokens, _ptr(q_nope), ld_qn, _ptr(q_pe), ld_qp,
+                                          _ptr(w_uk), _ptr(q_pos), _ptr(rope_table), max_pos, T,
+                                          n_h, _ptr(q_full), _ptr(status), _stream(stream)),
+           "mla_append_fp8_absorb_q")
 
 
 def mla_append_absorb_q(cache, num_pages, block_table, batch, max_pages, seq_idx, tok_pos, c_kv,

@@ -60,8 +60,10 @@ class _GraphStep:
 class DecodeSession(_GraphStep):
     """One attention-only decode step per call of ``step()``:
 
-        mla_cache_append (RoPE on the new keys, paged scatter)
-        mla_absorb_q     (q~ = q^C W^UK, RoPE on q^R, pack [q~ | q^R])
+        mla_append_absorb_q (mla_append_fp8_absorb_q with the FP8 cache):
+            the cache append (RoPE on the new keys, paged scatter) and the
+            absorption (q~ = q^C W^UK, RoPE on q^R, pack [q~ | q^R]) in one
+            launch
         mla_decode_attention (split-KV attention + combine)
         mla_out_absorb   (u = W^UV o)
     """
@@ -173,7 +175,15 @@ class DecodeSession(_GraphStep):
         mla.mla_out_absorb(self.o, self.w_uv, self.T, self.n_h, self.u, self.n_h * D_V, stream)
 
     def append_absorb(self, stream=None):
-        """append + absorb in one launch (the bf16 cache)."""
+        """append + absorb in one launch."""
+        if self.fp8:
+            mla.mla_append_fp8_absorb_q(self.cache8, self.scales8, self.num_pages, self.table,
+                                        self.B, self.max_pages, self.seq_idx, self.pos,
+                                        self.c_new, D_C, self.k_new, D_R, self.T, self.q_nope,
+                                        self.n_h * D_NOPE, self.q_pe, self.n_h * D_R, self.w_uk,
+                                        self.pos, self.rope, self.max_pos, self.T, self.n_h,
+                                        self.q_full, self.status, stream)
+            return
         mla.mla_append_absorb_q(self.cache, self.num_pages, self.table, self.B, self.max_pages,
                                 self.seq_idx, self.pos, self.c_new, D_C, self.k_new, D_R, self.T,
                                 self.q_nope, self.n_h * D_NOPE, self.q_pe, self.n_h * D_R,
@@ -181,11 +191,7 @@ class DecodeSession(_GraphStep):
                                 self.q_full, self.status, stream)
 
     def step(self, stream=None):
-        if self.fp8:
-            self.append(stream)
-            self.absorb(stream)
-        else:
-            self.append_absorb(stream)
+        self.append_absorb(stream)
         self.attend(stream)
         self.expand(stream)
 

@@ -79,6 +79,9 @@ def test_empty_inputs_are_noops_without_a_device(lib):
     # the fused append + absorption with neither tokens to append nor queries
     mla.mla_append_absorb_q(None, 1, None, 1, 1, None, None, None, 576, None, 576, 0, None, 24576,
                             None, 24576, None, None, None, 1, 0, 128, None, stream=0)
+    mla.mla_append_fp8_absorb_q(None, None, 1, None, 1, 1, None, None, None, 576, None, 576, 0,
+                                None, 24576, None, 24576, None, None, None, 1, 0, 128, None,
+                                stream=0)
     # the FP8 cache's entry points, the folds and the folded absorption
     mla.mla_cache_append_fp8(None, None, 1, None, 1, 1, None, None, None, 512, None, 64, None, 1,
                              0, stream=0)
@@ -103,6 +106,11 @@ def test_fused_append_absorb_checks_both_halves(lib):
         mla.mla_append_absorb_q(None, 1, None, 1, 1, None, None, None, 576, None, 576, 0, 16,
                                 2048, 16, 1024, 16, None, None, 0, 1, 24, 16, stream=0)
     assert e.value.status == mla.MLA_ERR_UNSUPPORTED
+    # the FP8 flavour: a NULL scale array with tokens to append
+    with pytest.raises(mla.MlaError) as e:
+        mla.mla_append_fp8_absorb_q(16, None, 1, 16, 1, 1, 16, 16, 16, 512, 16, 64, 4, 16, 16384,
+                                    16, 8192, 16, None, 16, 1, 1, 128, 16, stream=0)
+    assert e.value.status == mla.MLA_ERR_INVALID_ARGUMENT
 
 
 def test_rope_table_matches_oracle(lib):
