@@ -82,3 +82,25 @@ def test_stored_traffic_figures_are_plausible():
         cache_bytes = 64 * 4096 * row[cache]
         assert cache_bytes <= t <= math.ceil(1.1 * cache_bytes) + out_bytes
     assert (bench.decode_sources_hash(), "v3", "bf16") in bench.TRAFFIC
+
+
+def test_reference_arm_line_on_the_host():
+    # `bench.py --impl reference` times the oracle on the host cores and
+    # prints one JSON line in the contract's shape (its own impl tag, the
+    # oracle as cpu_baseline, an e2e object with no host<->device bytes)
+    import json
+    import subprocess
+    import sys
+    out = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--workload", "tiny",
+                          "--steps", "2", "--warmup", "1"], capture_output=True, text=True,
+                         timeout=300, cwd=bench.ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [l for l in out.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC and d["unit"] == bench.UNIT
+    assert d["value"] > 0 and d["higher_is_better"] is True and d["steps"] == 2
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["cpu_baseline"]["cores"] >= 1 and d["cpu_baseline"]["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
